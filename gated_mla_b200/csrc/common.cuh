@@ -1,0 +1,104 @@
+// common.cuh — types shared by the kernels and the C-ABI layer.
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace gmla {
+
+// Latent cache as the kernels see it (rows of `row` elements).
+struct CacheView {
+  void* data;
+  const int32_t* block_table;
+  int32_t paged;
+  int32_t batch;
+  int32_t capacity;
+  int32_t page_size;
+  int32_t num_pages;
+  int32_t max_pages_per_seq;
+  int32_t row;          // d_c + d_R
+};
+
+// Global row index of token `pos` of sequence `b`, or -1 when out of range.
+__device__ __forceinline__ int64_t cache_row(const CacheView& c, int b, int pos) {
+  if (b < 0 || pos < 0) return -1;
+  if (!c.paged) {
+    if (b >= c.batch || pos >= c.capacity) return -1;
+    return static_cast<int64_t>(b) * c.capacity + pos;
+  }
+  const int pi = pos / c.page_size;
+  if (b >= c.batch || pi >= c.max_pages_per_seq) return -1;
+  const int page = c.block_table[static_cast<int64_t>(b) * c.max_pages_per_seq + pi];
+  if (page < 0 || page >= c.num_pages) return -1;
+  return static_cast<int64_t>(page) * c.page_size + (pos % c.page_size);
+}
+
+// How a GEMM epilogue writes one weight segment's outputs.
+// Element (token t, feature f) goes to
+//   out + row(t) * row_stride + (f / block) * block_stride + (f % block) + col_offset
+// where row(t) = t, or the cache row of (seq_ids[t], positions[t]) when
+// `cache_scatter` is set. With `rope`, features (2i, 2i+1) of each block are
+// rotated by positions[t] * base^(-2i/block) first.
+struct EpiSeg {
+  void* out;
+  const float* bias;     // fp32 [rows] or null
+  int64_t row_stride;
+  int32_t block;
+  int32_t block_stride;
+  int32_t col_offset;
+  int32_t out_f32;       // 1: fp32 output, 0: bf16 output
+  int32_t rope;
+  int32_t cache_scatter;
+};
+
+constexpr int kMaxSeg = 5;
+
+struct GemmArgs {
+  CUtensorMap act;               // [T rows, K] bf16, box {64, token tile}
+  CUtensorMap wt[kMaxSeg];       // per segment [rows, K] bf16, box {64, weight tile}
+  EpiSeg epi[kMaxSeg];
+  int32_t seg_rows[kMaxSeg];
+  int32_t seg_tile_begin[kMaxSeg + 1];
+  int32_t n_seg;
+  int32_t T;
+  int32_t K;
+  // row_mode 0: token tile y covers packed tokens [y*tile, ...).
+  // row_mode 1: prefill sequence tiles: y -> (sequence y / tiles_per_seq,
+  //   offset (y % tiles_per_seq) * tile); activation rows start at
+  //   sequence * act_seq_stride, packed tokens at cu_seqlens[sequence].
+  int32_t row_mode;
+  int32_t tiles_per_seq;
+  int32_t act_seq_stride;
+  const int32_t* cu_seqlens;
+  const int32_t* positions;
+  const int32_t* seq_ids;
+  CacheView cache;
+  double log2_rope_base;
+  int* status;
+};
+
+// RoPE of one element given its pair partner: pair (x0, x1) at feature
+// (2i, 2i+1) becomes (x0 cos - x1 sin, x0 sin + x1 cos), angle pos * base^(-2i/d).
+// The angle is formed and reduced in double so long positions keep their accuracy.
+__device__ __forceinline__ float rope_rotate(float v, float partner, bool odd, int pos, int i_pair, int d,
+                                             double log2_base) {
+  const double inv = exp2(-(2.0 * i_pair / d) * log2_base);
+  double ang = static_cast<double>(pos) * inv;
+  ang -= 6.283185307179586476925 * rint(ang * 0.159154943091895335768883763);
+  float s, c;
+  sincosf(static_cast<float>(ang), &s, &c);
+  return odd ? (partner * s + v * c) : (v * c - partner * s);
+}
+
+__device__ __forceinline__ void epi_store(const EpiSeg& e, int64_t row, int f, float v) {
+  const int64_t off = row * e.row_stride + static_cast<int64_t>(f / e.block) * e.block_stride + (f % e.block) +
+                      e.col_offset;
+  if (e.bias) v += e.bias[f];
+  if (e.out_f32)
+    static_cast<float*>(e.out)[off] = v;
+  else
+    static_cast<__nv_bfloat16*>(e.out)[off] = __float2bfloat16_rn(v);
+}
+
+}  // namespace gmla

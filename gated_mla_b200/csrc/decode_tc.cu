@@ -1,0 +1,701 @@
+// decode_tc.cu — absorbed-form Gated MLA decode on tcgen05 tensor cores.
+//
+// The method ("Gated MLA 计算公式" §一/§二, "精读笔记 03" §5.1, §5.2, 题4):
+//   q_lat^(h) = W_k^(h)T q^(h)                      (absorption of W_k into the query)
+//   z_s       = scale * (q_lat^(h) . c_s + q^R(h) . k^R_s),   s < L
+//   O_lat     = sum_s softmax(z)_s c_s              (weighted sum in latent space)
+//   o^(h)     = W_v^(h) O_lat;   out = sigmoid(g) ⊙ o   (W_v absorbed on the output side)
+//
+// Kernels, in launch order:
+//   1. decode_plan      split the cached tokens of all sequences into equal
+//                       per-CTA ranges of 128-token tiles (segments).
+//   2. decode_absorb    q_lat = W_k^T q (times scale*log2 e), bf16, with q^R appended.
+//   3. decode_attn      per (CTA range, head group): TMA streams the latent rows
+//                       through a ring of 16 KB boxes; tcgen05 computes
+//                       S^T = C Q_lat^T (M = 128 tokens, N = heads) into TMEM; four
+//                       softmax warps turn S^T into P (online softmax, fp32,
+//                       rescaling only when a running max grows by > 2^8); tcgen05
+//                       accumulates O^T = C^T P^T (M = 128 latent dims, N = heads)
+//                       in TMEM; at a segment end the partial (O, m, l) goes out.
+//   4. decode_merge     merges the partials of each (sequence, head) by their
+//                       log-sum-exp weights, applies W_v and the sigmoid gate and
+//                       writes the gated head outputs once.
+#include "common.cuh"
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace gmla {
+
+constexpr int kTileTok = 128;   // tokens per tile (MMA M of S^T)
+constexpr int kBoxBytes = 128 * 128;   // one box: 128 token rows x 64 bf16
+constexpr int kDc = 512;        // latent width handled by the tensor-core path
+constexpr int kNcBox = kDc / 64;
+
+// ---------------------------------------------------------------------------
+// 1. plan
+// ---------------------------------------------------------------------------
+// Exclusive prefix sum over a block of 1024 threads; *total gets the sum.
+__device__ __forceinline__ int block_excl_scan_1024(int v, int* s_warp, int* total) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  int inc = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += n;
+  }
+  if (lane == 31) s_warp[w] = inc;
+  __syncthreads();
+  if (w == 0) {
+    const int x = s_warp[lane];
+    int y = x;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, y, o);
+      if (lane >= o) y += n;
+    }
+    s_warp[lane] = y - x;
+    if (lane == 31) *total = y;
+  }
+  __syncthreads();
+  const int r = s_warp[w] + inc - v;
+  __syncthreads();
+  return r;
+}
+
+// Tiles of 128 tokens of all sequences, concatenated, are cut into G equal
+// ranges (one per CTA of a head group). A segment is the part of one sequence
+// inside one range; seg_info = {sequence, first tile, end tile, CTA}.
+__global__ void __launch_bounds__(1024) decode_plan_kernel(DecodeArgs a) {
+  __shared__ int s_warp[32];
+  __shared__ int s_total;
+  __shared__ int s_sum;
+  const int tid = threadIdx.x;
+  const int limit = a.cache.paged ? a.cache.max_pages_per_seq * a.cache.page_size : a.cache.capacity;
+  if (tid == 0) s_sum = 0;
+  __syncthreads();
+  for (int b = tid; b < a.B; b += blockDim.x) {
+    int L = a.seq_lens[b];
+    if (L < 0 || L > limit || b >= a.cache.batch) {
+      report_status(a.status, kStatusRange);
+      L = 0;
+    }
+    atomicAdd(&s_sum, (L + kTileTok - 1) / kTileTok);
+  }
+  __syncthreads();
+  const int total = s_sum;
+  const int tpc = total > 0 ? (total + a.G - 1) / a.G : 1;
+  int tile_carry = 0, seg_carry = 0;
+  for (int base = 0; base < a.B; base += blockDim.x) {
+    const int b = base + tid;
+    int L = b < a.B ? a.seq_lens[b] : 0;
+    if (L < 0 || L > limit || b >= a.cache.batch) L = 0;
+    const int t = (L + kTileTok - 1) / kTileTok;
+    int tsum, ssum;
+    const int P = tile_carry + block_excl_scan_1024(t, s_warp, &s_total);
+    tsum = s_total;
+    int nseg = 0, g_first = 0;
+    if (t > 0) {
+      g_first = P / tpc;
+      nseg = (P + t - 1) / tpc - g_first + 1;
+    }
+    const int S = seg_carry + block_excl_scan_1024(nseg, s_warp, &s_total);
+    ssum = s_total;
+    if (b < a.B) {
+      a.seq_first_seg[b] = S;
+      for (int k = 0; k < nseg; ++k) {
+        const int g = g_first + k;
+        const int lo = max(P, g * tpc), hi = min(P + t, (g + 1) * tpc);
+        a.seg_info[S + k] = make_int4(b, lo - P, hi - P, g);
+        if (g * tpc >= P) a.cta_first_seg[g] = S + k;   // range g starts inside sequence b
+      }
+    }
+    tile_carry += tsum;
+    seg_carry += ssum;
+  }
+  if (tid == 0) a.seq_first_seg[a.B] = seg_carry;
+  const int g_used = total > 0 ? (total - 1) / tpc + 1 : 0;
+  for (int g = g_used + tid; g <= a.G; g += blockDim.x) a.cta_first_seg[g] = seg_carry;
+}
+
+// ---------------------------------------------------------------------------
+// 2. absorb: qa[b, h, :d_c] = bf16(q_scale * W_k^(h)T q^(h)), qa[b, h, d_c:] = bf16(q_scale * q^R)
+// ---------------------------------------------------------------------------
+constexpr int kAbsorbB = 8;
+
+__global__ void __launch_bounds__(128) decode_absorb_kernel(DecodeArgs a) {
+  const int h = blockIdx.x;
+  const int b0 = blockIdx.y * kAbsorbB;
+  const int nb = min(kAbsorbB, a.B - b0);
+  const int dq = a.d_h + a.d_rope;
+  const int row = a.d_c + a.d_rope;
+  extern __shared__ float sq[];   // [kAbsorbB][d_h]
+  const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(a.q);
+  for (int i = threadIdx.x; i < kAbsorbB * a.d_h; i += blockDim.x) {
+    const int bi = i / a.d_h, k = i % a.d_h;
+    sq[i] = bi < nb ? __bfloat162float(q[(static_cast<int64_t>(b0 + bi) * a.H + h) * dq + k]) : 0.f;
+  }
+  __syncthreads();
+  const __nv_bfloat16* Wk = static_cast<const __nv_bfloat16*>(a.W_k) + static_cast<int64_t>(h) * a.d_h * a.d_c;
+  __nv_bfloat16* qa = static_cast<__nv_bfloat16*>(a.qa);
+  // each thread: 4 consecutive latent columns
+  for (int c0 = threadIdx.x * 4; c0 < a.d_c; c0 += blockDim.x * 4) {
+    float acc[kAbsorbB][4];
+#pragma unroll
+    for (int bi = 0; bi < kAbsorbB; ++bi)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[bi][j] = 0.f;
+    for (int k = 0; k < a.d_h; ++k) {
+      const uint2 wv = *reinterpret_cast<const uint2*>(Wk + static_cast<int64_t>(k) * a.d_c + c0);
+      const __nv_bfloat162 w01 = *reinterpret_cast<const __nv_bfloat162*>(&wv.x);
+      const __nv_bfloat162 w23 = *reinterpret_cast<const __nv_bfloat162*>(&wv.y);
+      const float w[4] = {__low2float(w01), __high2float(w01), __low2float(w23), __high2float(w23)};
+#pragma unroll
+      for (int bi = 0; bi < kAbsorbB; ++bi) {
+        const float qk = sq[bi * a.d_h + k];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[bi][j] = fmaf(qk, w[j], acc[bi][j]);
+      }
+    }
+#pragma unroll
+    for (int bi = 0; bi < kAbsorbB; ++bi) {
+      if (bi >= nb) break;
+      __nv_bfloat16* dst = qa + (static_cast<int64_t>(b0 + bi) * a.H + h) * row + c0;
+      uint2 pk;
+      pk.x = pack_bf16x2(acc[bi][0] * a.q_scale, acc[bi][1] * a.q_scale);
+      pk.y = pack_bf16x2(acc[bi][2] * a.q_scale, acc[bi][3] * a.q_scale);
+      *reinterpret_cast<uint2*>(dst) = pk;
+    }
+  }
+  // decoupled RoPE query dims: copied (already rotated), scaled
+  for (int i = threadIdx.x; i < nb * a.d_rope; i += blockDim.x) {
+    const int bi = i / a.d_rope, r = i % a.d_rope;
+    const int64_t src = (static_cast<int64_t>(b0 + bi) * a.H + h) * dq + a.d_h + r;
+    qa[(static_cast<int64_t>(b0 + bi) * a.H + h) * row + a.d_c + r] =
+        __float2bfloat16_rn(__bfloat162float(q[src]) * a.q_scale);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// 3. attention over the latent cache
+// ---------------------------------------------------------------------------
+struct DecSmem {
+  uint64_t full[12], empty[12];
+  uint64_t rope_full, rope_empty;
+  uint64_t q_full, q_empty;
+  uint64_t s_full, p_full, o_done, o_free, drain;
+  uint32_t tmem;
+  int abort;
+  int vote[2];
+  int red[2][4][64];
+  float lred[4][64];
+};
+
+template <int HG, int NBOX>
+struct DecCfg {
+  static constexpr bool kRope = NBOX > kNcBox;
+  static constexpr int kQBytes = NBOX * HG * 128;          // absorbed queries, NBOX boxes of [HG x 64]
+  static constexpr int kPBytes = kRope ? 0 : HG * 256;     // P [HG x 128] (K-major, 2 blocks); rope slot otherwise
+  static constexpr int kRopeBytes = kRope ? kBoxBytes : 0;
+  static constexpr int kSmemStruct = (static_cast<int>(sizeof(DecSmem)) + 127) & ~127;
+  static constexpr int kFixed = kQBytes + kPBytes + kRopeBytes + kSmemStruct + 1024 /*align*/;
+  static constexpr int kBudget = 232448;
+  static constexpr int kRingMax = (kBudget - kFixed) / kBoxBytes;
+  static constexpr int kRing = (kRingMax > 12 ? 12 : kRingMax) & ~1;   // even: box pairs never wrap
+  static constexpr int kSmem = kRing * kBoxBytes + kFixed;
+  static constexpr int kTmemCols = (5 * HG <= 128) ? 128 : ((5 * HG <= 256) ? 256 : 512);
+  static_assert(kRing >= kNcBox, "ring must hold one tile");
+};
+
+template <int HG, int NBOX>
+__global__ void __launch_bounds__(192, 1) decode_attn_kernel(const __grid_constant__ DecodeArgs a) {
+  using C = DecCfg<HG, NBOX>;
+  constexpr int NR = C::kRing;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* ring = smem;
+  uint8_t* rope_slot = ring + NR * kBoxBytes;
+  uint8_t* qs = rope_slot + C::kRopeBytes;
+  uint8_t* pbuf = C::kRope ? rope_slot : (qs + C::kQBytes);
+  DecSmem* sm = reinterpret_cast<DecSmem*>(qs + C::kQBytes + C::kPBytes);
+  volatile int* abort_flag = &sm->abort;
+
+  const int g = blockIdx.x, hg = blockIdx.y;
+  const int seg_lo = a.cta_first_seg[g], seg_hi = a.cta_first_seg[g + 1];
+  if (seg_lo >= seg_hi) return;   // uniform: no work for this CTA
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int heads_valid = min(HG, a.H - hg * HG);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NR; ++i) {
+      mbar_init(&sm->full[i], 1);
+      mbar_init(&sm->empty[i], 1);
+    }
+    mbar_init(&sm->rope_full, 1);
+    mbar_init(&sm->rope_empty, 1);
+    mbar_init(&sm->q_full, 1);
+    mbar_init(&sm->q_empty, 1);
+    mbar_init(&sm->s_full, 1);
+    mbar_init(&sm->p_full, 128);
+    mbar_init(&sm->o_done, 1);
+    mbar_init(&sm->o_free, 128);
+    mbar_init(&sm->drain, 1);
+    sm->abort = 0;
+    sm->vote[0] = sm->vote[1] = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&sm->tmem, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm->tmem;
+  const uint32_t tS = tmem;          // S^T: HG columns
+  const uint32_t tO = tmem + HG;     // O^T: kNcBox/2 chunks of HG columns
+
+  if (warp == 0) {
+    // ------------------------------ TMA producer ------------------------------
+    if (lane == 0) {
+      tma_prefetch_desc(&a.cache_map);
+      tma_prefetch_desc(&a.qa_map);
+      const uint64_t pol_c = a.n_hg > 1 ? l2_evict_normal() : l2_evict_first();
+      const uint64_t pol_q = l2_evict_last();
+      uint32_t nbox = 0, nrope = 0, nq = 0;
+      bool ok = true;
+      for (int si = seg_lo; si < seg_hi && ok; ++si) {
+        const int4 sg = a.seg_info[si];
+        const int b = sg.x;
+        const int L = a.seq_lens[b];
+        if (nq > 0 && !mbar_wait(&sm->q_empty, (nq - 1) & 1, abort_flag, a.status)) { ok = false; break; }
+        mbar_arrive_expect_tx(&sm->q_full, C::kQBytes);
+        for (int j = 0; j < NBOX; ++j)
+          tma_load_2d(&a.qa_map, &sm->q_full, qs + j * HG * 128, j * 64, b * a.H + hg * HG, pol_q);
+        ++nq;
+        for (int t = sg.y; t < sg.z && ok; ++t) {
+          const int tok0 = t * kTileTok;
+          const int valid = min(kTileTok, L - tok0);
+          for (int j = 0; j < NBOX; ++j) {
+            uint64_t* bar;
+            uint8_t* dst;
+            if (j < kNcBox) {
+              const uint32_t slot = nbox % NR;
+              if (nbox >= static_cast<uint32_t>(NR) &&
+                  !mbar_wait(&sm->empty[slot], ((nbox / NR) & 1) ^ 1, abort_flag, a.status)) { ok = false; break; }
+              bar = &sm->full[slot];
+              dst = ring + slot * kBoxBytes;
+              ++nbox;
+            } else {
+              if (nrope > 0 && !mbar_wait(&sm->rope_empty, (nrope - 1) & 1, abort_flag, a.status)) { ok = false; break; }
+              bar = &sm->rope_full;
+              dst = rope_slot;
+              ++nrope;
+            }
+            if (!a.cache.paged) {
+              mbar_arrive_expect_tx(bar, kBoxBytes);
+              tma_load_2d(&a.cache_map, bar, dst, j * 64, b * a.cache.capacity + tok0, pol_c);
+            } else {
+              const int ps = a.cache.page_size;
+              const int32_t* bt = a.cache.block_table + static_cast<int64_t>(b) * a.cache.max_pages_per_seq;
+              if (ps >= kTileTok) {
+                mbar_arrive_expect_tx(bar, kBoxBytes);
+                tma_load_3d(&a.cache_map, bar, dst, j * 64, tok0 % ps, bt[tok0 / ps], pol_c);
+              } else {
+                const int nchunk = (valid + ps - 1) / ps;
+                mbar_arrive_expect_tx(bar, nchunk * ps * 128);
+                for (int r = 0; r < nchunk; ++r)
+                  tma_load_3d(&a.cache_map, bar, dst + r * ps * 128, j * 64, 0, bt[(tok0 + r * ps) / ps], pol_c);
+              }
+            }
+          }
+        }
+      }
+      if (*abort_flag) {   // let issued copies land before the block exits
+        for (uint32_t c = nbox > static_cast<uint32_t>(NR) ? nbox - NR : 0; c < nbox; ++c)
+          mbar_drain(&sm->full[c % NR], (c / NR) & 1);
+        if (nrope) mbar_drain(&sm->rope_full, (nrope - 1) & 1);
+        if (nq) mbar_drain(&sm->q_full, (nq - 1) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------ MMA issuer ------------------------------
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16_f32(128, HG, false, false);
+      constexpr uint32_t idO = idesc_bf16_f32(128, HG, true, false);
+      const uint32_t ring_a = smem_u32(ring), rope_a = smem_u32(rope_slot), q_a = smem_u32(qs),
+                     p_a = smem_u32(pbuf);
+      uint32_t nbox = 0, nrope = 0, ntile = 0, nseg = 0;
+      bool ok = true;
+      for (int si = seg_lo; si < seg_hi && ok; ++si, ++nseg) {
+        const int4 sg = a.seg_info[si];
+        if (!mbar_wait(&sm->q_full, nseg & 1, abort_flag, a.status)) { ok = false; break; }
+        for (int t = sg.y; t < sg.z; ++t, ++ntile) {
+          // S^T = C Q^T
+          for (int j = 0; j < NBOX; ++j) {
+            uint32_t sa;
+            if (j < kNcBox) {
+              const uint32_t c = nbox + j, slot = c % NR;
+              if (!mbar_wait(&sm->full[slot], (c / NR) & 1, abort_flag, a.status)) { ok = false; break; }
+              sa = ring_a + slot * kBoxBytes;
+            } else {
+              if (!mbar_wait(&sm->rope_full, nrope & 1, abort_flag, a.status)) { ok = false; break; }
+              sa = rope_a;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              umma_bf16(tS, sdesc_sw128(sa + kk * 32, 16, 1024),
+                        sdesc_sw128(q_a + j * HG * 128 + kk * 32, 16, 1024), idS, (j | kk) != 0);
+          }
+          if (!ok) break;
+          if (t + 1 == sg.z) umma_commit(&sm->q_empty);
+          umma_commit(&sm->s_full);
+          // wait for P, then O^T += C^T P^T
+          if (!mbar_wait(&sm->p_full, ntile & 1, abort_flag, a.status)) { ok = false; break; }
+          const bool first = (t == sg.y);
+          if (first && nseg > 0 && !mbar_wait(&sm->o_free, (nseg - 1) & 1, abort_flag, a.status)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll 1
+          for (int mc = 0; mc < kNcBox / 2; ++mc) {
+            const uint32_t c0 = nbox + 2 * mc, slot0 = c0 % NR;
+            const uint32_t sa = ring_a + slot0 * kBoxBytes;
+#pragma unroll
+            for (int kk = 0; kk < kTileTok / 16; ++kk) {
+              const uint64_t ad = sdesc_sw128(sa + kk * 2048, kBoxBytes, 1024);
+              const uint64_t bd = sdesc_sw128(p_a + (kk >> 2) * (HG * 128) + (kk & 3) * 32, 16, 1024);
+              umma_bf16(tO + mc * HG, ad, bd, idO, (!first || kk > 0) ? 1u : 0u);
+            }
+            umma_commit(&sm->empty[slot0]);
+            umma_commit(&sm->empty[slot0 + 1]);
+          }
+          if (C::kRope) umma_commit(&sm->rope_empty);
+          nbox += kNcBox;
+          if (C::kRope) ++nrope;
+        }
+        if (!ok) break;
+        umma_commit(&sm->o_done);
+      }
+      if (!ok) {
+        umma_commit(&sm->drain);
+        mbar_drain(&sm->drain, 0);
+      }
+    }
+  } else {
+    // ------------------------------ softmax warps ------------------------------
+    const int q4 = warp & 3;
+    const int row = q4 * 32 + lane;                      // token row of the tile / latent row of a chunk
+    const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
+    const int ltid = threadIdx.x - 64;                   // 0..127
+    const float NEG_INF = -__int_as_float(0x7f800000);
+    // The four softmax warps meet at named barrier 1. After a failed wait a
+    // warp keeps walking the same loops (skipping the waits) so every warp
+    // executes the same sequence of barriers and the block can exit.
+    uint32_t nbox = 0, ntile = 0, nseg = 0;
+    bool ok = true;
+    for (int si = seg_lo; si < seg_hi; ++si, ++nseg) {
+      const int4 sg = a.seg_info[si];
+      const int L = a.seq_lens[sg.x];
+      float m[HG], lsum[HG];
+#pragma unroll
+      for (int h = 0; h < HG; ++h) {
+        m[h] = NEG_INF;
+        lsum[h] = 0.f;
+      }
+      for (int t = sg.y; t < sg.z; ++t, ++ntile) {
+        const bool first = (t == sg.y);
+        ok = ok && mbar_wait(&sm->s_full, ntile & 1, abort_flag, a.status);
+        tc_fence_after();
+        float s[HG];
+#pragma unroll
+        for (int c = 0; c < HG; c += 16) {
+          uint32_t v[16];
+          tmem_ld16(tS + lane_off + c, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) s[c + j] = __uint_as_float(v[j]);
+        }
+        const int valid = min(kTileTok, L - t * kTileTok);
+        const bool rv = row < valid;
+        bool need = first;
+#pragma unroll
+        for (int h = 0; h < HG; ++h) {
+          if (!rv) s[h] = NEG_INF;
+          need |= s[h] > m[h] + 8.f;
+        }
+        // block-wide vote among the 128 softmax threads
+        const int par = ntile & 1;
+        if (__any_sync(0xffffffffu, need) && lane == 0) atomicOr(&sm->vote[par], 1);
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        const bool need_all = sm->vote[par] != 0;
+        if (ltid == 0) sm->vote[par ^ 1] = 0;
+        if (need_all) {
+#pragma unroll
+          for (int h = 0; h < HG; ++h) {
+            const int k = __reduce_max_sync(0xffffffffu, float_to_ordered(s[h]));
+            if (lane == 0) sm->red[par][q4][h] = k;
+          }
+          asm volatile("bar.sync 1, 128;" ::: "memory");
+          float alpha[HG];
+          bool rescale = false;
+#pragma unroll
+          for (int h = 0; h < HG; ++h) {
+            int k = sm->red[par][0][h];
+            k = max(k, sm->red[par][1][h]);
+            k = max(k, sm->red[par][2][h]);
+            k = max(k, sm->red[par][3][h]);
+            const float tmax = ordered_to_float(k);
+            const float mn = fmaxf(m[h], tmax);
+            alpha[h] = (m[h] == NEG_INF) ? 0.f : ex2_approx(m[h] - mn);
+            rescale |= (mn > m[h]) && !first;
+            m[h] = mn;
+            lsum[h] *= alpha[h];
+          }
+          if (rescale) {
+            // O^T columns of head h scale by alpha[h] (O of the previous tile is complete:
+            // S of this tile was issued after it)
+#pragma unroll 1
+            for (int mc = 0; mc < kNcBox / 2; ++mc) {
+#pragma unroll
+              for (int c = 0; c < HG; c += 16) {
+                uint32_t v[16];
+                tmem_ld16(tO + lane_off + mc * HG + c, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 16; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * alpha[c + j]);
+                tmem_st16(tO + lane_off + mc * HG + c, v);
+              }
+            }
+            tmem_st_wait();
+          }
+        }
+        // P = exp2(s - m), stored bf16 as P[h][token] (K-major B operand, 2 blocks of 64 tokens)
+        uint8_t* pb = pbuf + (row >> 6) * (HG * 128);
+        const int pc = row & 63;
+#pragma unroll
+        for (int h = 0; h < HG; ++h) {
+          const float p = rv ? ex2_approx(s[h] - m[h]) : 0.f;
+          lsum[h] += p;
+          *reinterpret_cast<__nv_bfloat16*>(pb + sw128_offset(h, pc)) = __float2bfloat16_rn(p);
+        }
+        if (!rv) {
+          // rows past the sequence end may hold anything: zero them so 0 * garbage cannot reach O
+#pragma unroll 1
+          for (int j = 0; j < kNcBox; ++j) {
+            uint8_t* box = ring + ((nbox + j) % NR) * kBoxBytes + row * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) reinterpret_cast<uint4*>(box)[c] = make_uint4(0, 0, 0, 0);
+          }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&sm->p_full);
+        nbox += kNcBox;
+      }
+      // ---- segment end: write the partial (unnormalised O, running max m, sum l)
+      ok = ok && mbar_wait(&sm->o_done, nseg & 1, abort_flag, a.status);
+      tc_fence_after();
+      const int par = nseg & 1;
+      (void)par;
+#pragma unroll
+      for (int h = 0; h < HG; ++h) {
+        float v = lsum[h];
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (lane == 0) sm->lred[q4][h] = v;
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      const int64_t pbase = (static_cast<int64_t>(hg) * a.max_seg + si) * HG;
+      if (ok && ltid < heads_valid) {
+        float l = 0.f;
+        float mh = NEG_INF;
+#pragma unroll
+        for (int h = 0; h < HG; ++h)
+          if (h == ltid) mh = m[h];
+        for (int w = 0; w < 4; ++w) l += sm->lred[w][ltid];
+        a.ml_part[(pbase + ltid) * 2 + 0] = mh;
+        a.ml_part[(pbase + ltid) * 2 + 1] = l;
+      }
+#pragma unroll 1
+      for (int mc = 0; mc < kNcBox / 2; ++mc) {
+#pragma unroll
+        for (int c = 0; c < HG; c += 16) {
+          uint32_t v[16];
+          tmem_ld16(tO + lane_off + mc * HG + c, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            if (ok && c + j < heads_valid)
+              a.o_part[(pbase + c + j) * kDc + mc * 128 + row] = __uint_as_float(v[j]);
+          }
+        }
+      }
+      tc_fence_before();
+      asm volatile("bar.sync 1, 128;" ::: "memory");   // lred reuse
+      mbar_arrive(&sm->o_free);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// 4. merge partials, W_v up-projection, sigmoid gate
+// ---------------------------------------------------------------------------
+constexpr int kMergeB = 4;
+
+__global__ void __launch_bounds__(256) decode_merge_kernel(DecodeArgs a) {
+  const int h = blockIdx.x;
+  const int b0 = blockIdx.y * kMergeB;
+  const int nb = min(kMergeB, a.B - b0);
+  const int hg = h / a.HG, hl = h % a.HG;
+  __shared__ float olat[kMergeB][kDc];
+  __shared__ float mx_s[kMergeB];
+  __shared__ float inv_l[kMergeB];
+  const int tid = threadIdx.x;
+  const int64_t base = static_cast<int64_t>(hg) * a.max_seg;
+  // m = max_i m_i, l = sum_i 2^(m_i - m) l_i over the segments of each sequence
+  if (tid < 32 * kMergeB) {
+    const int bi = tid >> 5, ln = tid & 31;
+    if (bi < nb) {
+      const int b = b0 + bi;
+      const int s0 = a.seq_first_seg[b], s1 = a.seq_first_seg[b + 1];
+      float mx = -__int_as_float(0x7f800000);
+      for (int s = s0 + ln; s < s1; s += 32) mx = fmaxf(mx, a.ml_part[((base + s) * a.HG + hl) * 2]);
+      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      float l = 0.f;
+      for (int s = s0 + ln; s < s1; s += 32) {
+        const float* ml = a.ml_part + ((base + s) * a.HG + hl) * 2;
+        l += ex2_approx(ml[0] - mx) * ml[1];
+      }
+      for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+      if (ln == 0) {
+        mx_s[bi] = mx;
+        inv_l[bi] = (s1 > s0 && l > 0.f) ? 1.f / l : 0.f;
+      }
+    }
+  }
+  __syncthreads();
+  // O_lat = sum_i 2^(m_i - m) O_i / l
+  for (int i = tid; i < kMergeB * kDc; i += blockDim.x) {
+    const int bi = i / kDc, d = i % kDc;
+    float acc = 0.f;
+    if (bi < nb) {
+      const int b = b0 + bi;
+      const int s0 = a.seq_first_seg[b], s1 = a.seq_first_seg[b + 1];
+      for (int s = s0; s < s1; ++s) {
+        const float w = ex2_approx(a.ml_part[((base + s) * a.HG + hl) * 2] - mx_s[bi]);
+        acc = fmaf(w, a.o_part[((base + s) * a.HG + hl) * kDc + d], acc);
+      }
+      acc *= inv_l[bi];
+    }
+    olat[bi][d] = acc;
+  }
+  __syncthreads();
+  // o[b, h*d_h + i] = sum_d W_v[h, i, d] * olat[b, d]; one warp per output row i
+  const __nv_bfloat16* Wv = static_cast<const __nv_bfloat16*>(a.W_v) + static_cast<int64_t>(h) * a.d_h * kDc;
+  const int warp = tid >> 5, lane = tid & 31;
+  __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.o);
+  const int HD = a.H * a.d_h;
+  const int G = a.gate_mode == 0 ? HD : a.H;
+  for (int i = warp; i < a.d_h; i += blockDim.x / 32) {
+    float acc[kMergeB];
+#pragma unroll
+    for (int bi = 0; bi < kMergeB; ++bi) acc[bi] = 0.f;
+    const __nv_bfloat16* wr = Wv + static_cast<int64_t>(i) * kDc;
+#pragma unroll
+    for (int it = 0; it < kDc / 256; ++it) {
+      const int d0 = it * 256 + lane * 8;
+      const uint4 wv = *reinterpret_cast<const uint4*>(wr + d0);
+      const __nv_bfloat162* w2 = reinterpret_cast<const __nv_bfloat162*>(&wv);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float wa = __low2float(w2[k]), wb = __high2float(w2[k]);
+#pragma unroll
+        for (int bi = 0; bi < kMergeB; ++bi)
+          acc[bi] = fmaf(wa, olat[bi][d0 + 2 * k], fmaf(wb, olat[bi][d0 + 2 * k + 1], acc[bi]));
+      }
+    }
+#pragma unroll
+    for (int bi = 0; bi < kMergeB; ++bi)
+      for (int o = 16; o > 0; o >>= 1) acc[bi] += __shfl_xor_sync(0xffffffffu, acc[bi], o);
+    if (lane < nb) {
+      const int b = b0 + lane;
+      float v = 0.f;
+#pragma unroll
+      for (int bi = 0; bi < kMergeB; ++bi)
+        if (bi == lane) v = acc[bi];
+      if (a.gate_logits) {
+        const float z = a.gate_logits[static_cast<int64_t>(b) * G + (a.gate_mode == 0 ? h * a.d_h + i : h)];
+        v *= 1.f / (1.f + __expf(-z));
+      }
+      out[static_cast<int64_t>(b) * HD + h * a.d_h + i] = __float2bfloat16_rn(v);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+DecodeLayout decode_layout(int B, int H, int d_c, int d_rope, int num_sms) {
+  DecodeLayout L{};
+  L.HG = H <= 16 ? 16 : (H % 64 == 0 ? 64 : (H % 32 == 0 ? 32 : 16));
+  L.n_hg = (H + L.HG - 1) / L.HG;
+  L.G = num_sms / L.n_hg;
+  if (L.G < 1) L.G = 1;
+  L.max_seg = L.G + B + 1;
+  const size_t row = static_cast<size_t>(d_c + d_rope);
+  size_t off = 256;   // status word
+  L.off_qa = off;
+  off = align256(off + static_cast<size_t>(B) * H * row * 2 + 16 * row * 2 /* padded head rows */);
+  L.off_opart = off;
+  off = align256(off + static_cast<size_t>(L.n_hg) * L.max_seg * L.HG * kDc * 4);
+  L.off_ml = off;
+  off = align256(off + static_cast<size_t>(L.n_hg) * L.max_seg * L.HG * 2 * 4);
+  L.off_seg = off;
+  off = align256(off + static_cast<size_t>(L.max_seg) * sizeof(int4));
+  L.off_seqfirst = off;
+  off = align256(off + static_cast<size_t>(B + 1) * 4);
+  L.off_ctafirst = off;
+  off = align256(off + static_cast<size_t>(L.G + 1) * 4);
+  L.total = off;
+  return L;
+}
+
+template <int HG, int NBOX>
+static cudaError_t launch_attn(const DecodeArgs& a, cudaStream_t st) {
+  using C = DecCfg<HG, NBOX>;
+  auto k = decode_attn_kernel<HG, NBOX>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+  if (e != cudaSuccess) return e;
+  k<<<dim3(a.G, a.n_hg), 192, C::kSmem, st>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode_bf16(DecodeArgs& a, cudaStream_t st) {
+  decode_plan_kernel<<<1, 1024, 0, st>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  decode_absorb_kernel<<<dim3(a.H, (a.B + kAbsorbB - 1) / kAbsorbB), 128, kAbsorbB * a.d_h * sizeof(float), st>>>(a);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const int nbox = (a.d_c + a.d_rope) / 64;
+  switch (a.HG * 16 + nbox) {
+    case 16 * 16 + 8: e = launch_attn<16, 8>(a, st); break;
+    case 16 * 16 + 9: e = launch_attn<16, 9>(a, st); break;
+    case 32 * 16 + 8: e = launch_attn<32, 8>(a, st); break;
+    case 32 * 16 + 9: e = launch_attn<32, 9>(a, st); break;
+    case 64 * 16 + 8: e = launch_attn<64, 8>(a, st); break;
+    case 64 * 16 + 9: e = launch_attn<64, 9>(a, st); break;
+    default: return cudaErrorInvalidValue;
+  }
+  if (e != cudaSuccess) return e;
+  decode_merge_kernel<<<dim3(a.H, (a.B + kMergeB - 1) / kMergeB), 256, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace gmla

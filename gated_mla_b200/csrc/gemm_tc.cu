@@ -1,0 +1,300 @@
+// gemm_tc.cu — bf16 GEMM on tcgen05 tensor cores with fused epilogues.
+//
+// D = X W^T for an activation X [T, K] and a weight that is a list of up to
+// kMaxSeg segments W_s [rows_s, K] (all K-major, row-major [out, in]). Each
+// segment has its own epilogue (plain store, fp32 + bias, RoPE, scatter into
+// the latent cache). Used for:
+//   * x -> [c | k^R | q | q^R | gate logits]   ("Gated MLA 计算公式" §一/§二;
+//                                                "精读笔记 03" §5.2)
+//   * latent rows -> K^(h), V^(h) for prefill    ("Gated MLA 计算公式" §一)
+//   * gated o -> y = W_o (...)                    ("Gated MLA 计算公式" §二 boxed eq.)
+//
+// Two orientations share one kernel:
+//   kSwap = true  (few tokens): MMA M = 128 weight rows, N = BN tokens.
+//   kSwap = false (many tokens): MMA M = 128 token rows, N = BN weight rows.
+// Roles: warp 0 issues TMA loads into a ring of shared-memory stages, warp 1
+// allocates TMEM and one thread issues the MMAs, warps 2..5 drain the fp32
+// accumulator from TMEM and run the epilogue. Every wait is bounded.
+#include "common.cuh"
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace gmla {
+
+template <int BN>
+struct GemmCfg {
+  static constexpr int kABytes = 128 * 128;              // 128 rows x 64 bf16
+  static constexpr int kBBytes = BN * 128;               // BN rows x 64 bf16
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kStages = (BN >= 256) ? 4 : (BN >= 128 ? 6 : 8);
+  static constexpr int kTmemCols = BN < 32 ? 32 : BN;
+  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+};
+
+struct GemmTile {
+  int seg;       // weight segment
+  int wrow0;     // first weight row of the tile (segment-local)
+  int tok0;      // first token index (packed) of the tile
+  int act_row0;  // first activation row read by TMA
+  int ntok;      // valid tokens in this tile
+};
+
+template <int BN, bool kSwap>
+__device__ __forceinline__ bool gemm_tile(const GemmArgs& a, GemmTile& t) {
+  const int wt = blockIdx.x;
+  int s = 0;
+  while (s + 1 < a.n_seg && wt >= a.seg_tile_begin[s + 1]) ++s;
+  t.seg = s;
+  constexpr int kWTile = kSwap ? 128 : BN;
+  constexpr int kTTile = kSwap ? BN : 128;
+  t.wrow0 = (wt - a.seg_tile_begin[s]) * kWTile;
+  if (a.row_mode == 0) {
+    t.tok0 = blockIdx.y * kTTile;
+    t.act_row0 = t.tok0;
+    t.ntok = min(kTTile, a.T - t.tok0);
+  } else {
+    // prefill sequence tiles: token tile -> (sequence, offset)
+    const int b = blockIdx.y / a.tiles_per_seq;
+    const int t0 = (blockIdx.y % a.tiles_per_seq) * kTTile;
+    const int beg = a.cu_seqlens[b], len = a.cu_seqlens[b + 1] - beg;
+    t.tok0 = beg + t0;
+    t.act_row0 = b * a.act_seq_stride + t0;
+    t.ntok = min(kTTile, len - t0);
+  }
+  return t.ntok > 0;
+}
+
+template <int BN, bool kSwap>
+__global__ void __launch_bounds__(192, 1) gemm_bf16_tc_kernel(const __grid_constant__ GemmArgs a) {
+  using C = GemmCfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
+  uint64_t* empty = full + C::kStages;
+  uint64_t* acc_full = empty + C::kStages;
+  uint64_t* drain = acc_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  GemmTile tile;
+  if (!gemm_tile<BN, kSwap>(a, tile)) return;   // uniform across the block
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int num_kb = (a.K + 63) / 64;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::kStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const CUtensorMap* wmap = &a.wt[tile.seg];
+      tma_prefetch_desc(&a.act);
+      tma_prefetch_desc(wmap);
+      const uint64_t pol_w = l2_evict_normal();
+      const uint64_t pol_x = l2_evict_last();
+      int issued = 0;
+      for (int kb = 0; kb < num_kb; ++kb) {
+        const int st = kb % C::kStages;
+        if (kb >= C::kStages &&
+            !mbar_wait(&empty[st], ((kb / C::kStages) & 1) ^ 1, abort_flag, a.status))
+          break;
+        uint8_t* sa = smem + st * C::kStageBytes;
+        uint8_t* sb = sa + C::kABytes;
+        mbar_arrive_expect_tx(&full[st], C::kStageBytes);
+        if (kSwap) {
+          tma_load_2d(wmap, &full[st], sa, kb * 64, tile.wrow0, pol_w);
+          tma_load_2d(&a.act, &full[st], sb, kb * 64, tile.act_row0, pol_x);
+        } else {
+          tma_load_2d(&a.act, &full[st], sa, kb * 64, tile.act_row0, pol_x);
+          tma_load_2d(wmap, &full[st], sb, kb * 64, tile.wrow0, pol_w);
+        }
+        ++issued;
+      }
+      if (*abort_flag) {   // let copies still in flight land before the block exits
+        for (int kb = max(0, issued - C::kStages); kb < issued; ++kb)
+          mbar_drain(&full[kb % C::kStages], (kb / C::kStages) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, BN, false, false);
+      bool ok = true;
+      for (int kb = 0; kb < num_kb; ++kb) {
+        const int st = kb % C::kStages;
+        if (!mbar_wait(&full[st], (kb / C::kStages) & 1, abort_flag, a.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t sa = smem_u32(smem + st * C::kStageBytes);
+        const uint32_t sb = sa + C::kABytes;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          umma_bf16(tmem, sdesc_sw128(sa + kk * 32, 16, 1024), sdesc_sw128(sb + kk * 32, 16, 1024), idesc,
+                    (kb | kk) != 0);
+        }
+        umma_commit(&empty[st]);
+      }
+      if (ok) {
+        umma_commit(acc_full);
+      } else {
+        umma_commit(drain);
+        mbar_drain(drain, 0);
+      }
+    }
+  } else {
+    // epilogue warps 2..5 -> TMEM lane quarter (warp % 4)
+    const int q = warp & 3;
+    const int r = q * 32 + lane;            // accumulator row of this thread
+    if (mbar_wait(acc_full, 0, abort_flag, a.status)) {
+      tc_fence_after();
+      const EpiSeg& e = a.epi[tile.seg];
+      const int seg_rows = a.seg_rows[tile.seg];
+      if (kSwap) {
+        // row r = weight feature, columns = tokens
+        const int f = tile.wrow0 + r;
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN; c0 += 16) {
+          uint32_t v[16];
+          tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + c0, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int tl = c0 + j;
+            float val = __uint_as_float(v[j]);
+            const int tok = tile.tok0 + tl;
+            const bool tok_ok = tl < tile.ntok;
+            int pos = 0;
+            if (e.rope || e.cache_scatter) pos = tok_ok ? a.positions[tok] : 0;
+            if (e.rope) {
+              const float partner = __shfl_xor_sync(0xffffffffu, val, 1);
+              const int fi = f % e.block;
+              val = rope_rotate(val, partner, fi & 1, pos, fi >> 1, e.block, a.log2_rope_base);
+            }
+            if (!tok_ok || f >= seg_rows) continue;
+            int64_t row = tok;
+            if (e.cache_scatter) {
+              row = cache_row(a.cache, a.seq_ids[tok], pos);
+              if (row < 0) {
+                report_status(a.status, kStatusRange);
+                continue;
+              }
+            }
+            epi_store(e, row, f, val);
+          }
+        }
+      } else {
+        // row r = token, columns = weight features
+        const bool tok_ok = r < tile.ntok;
+        const int tok = tile.tok0 + r;
+        int pos = 0;
+        int64_t row = tok;
+        if (tok_ok && (e.rope || e.cache_scatter)) pos = a.positions[tok];
+        if (tok_ok && e.cache_scatter) {
+          row = cache_row(a.cache, a.seq_ids[tok], pos);
+          if (row < 0) report_status(a.status, kStatusRange);
+        }
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN; c0 += 16) {
+          uint32_t v[16];
+          tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + c0, v);
+          tmem_ld_wait();
+          if (!tok_ok || row < 0) continue;
+          const int f0 = tile.wrow0 + c0;
+          float x[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) x[j] = __uint_as_float(v[j]);
+          if (e.rope) {
+#pragma unroll
+            for (int j = 0; j < 16; j += 2) {
+              const int fi = (f0 + j) % e.block;
+              const float x0 = x[j], x1 = x[j + 1];
+              x[j] = rope_rotate(x0, x1, false, pos, fi >> 1, e.block, a.log2_rope_base);
+              x[j + 1] = rope_rotate(x1, x0, true, pos, fi >> 1, e.block, a.log2_rope_base);
+            }
+          }
+          const bool vec = !e.out_f32 && !e.bias && (f0 + 16 <= seg_rows) && (f0 % e.block) + 16 <= e.block &&
+                           ((row * e.row_stride + (f0 / e.block) * (int64_t)e.block_stride + (f0 % e.block) +
+                             e.col_offset) % 8 == 0);
+          if (vec) {
+            const int64_t off = row * e.row_stride + static_cast<int64_t>(f0 / e.block) * e.block_stride +
+                                (f0 % e.block) + e.col_offset;
+            uint4 p0, p1;
+            p0.x = pack_bf16x2(x[0], x[1]);
+            p0.y = pack_bf16x2(x[2], x[3]);
+            p0.z = pack_bf16x2(x[4], x[5]);
+            p0.w = pack_bf16x2(x[6], x[7]);
+            p1.x = pack_bf16x2(x[8], x[9]);
+            p1.y = pack_bf16x2(x[10], x[11]);
+            p1.z = pack_bf16x2(x[12], x[13]);
+            p1.w = pack_bf16x2(x[14], x[15]);
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(e.out) + off);
+            dst[0] = p0;
+            dst[1] = p1;
+          } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              if (f0 + j < seg_rows) epi_store(e, row, f0 + j, x[j]);
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+template <int BN, bool kSwap>
+static cudaError_t launch_one(const GemmArgs& a, dim3 grid, cudaStream_t st) {
+  using C = GemmCfg<BN>;
+  auto k = gemm_bf16_tc_kernel<BN, kSwap>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  k<<<grid, 192, C::kSmemBytes, st>>>(a);
+  return cudaGetLastError();
+}
+
+int gemm_weight_tile(bool swap, int bn) { return swap ? 128 : bn; }
+
+cudaError_t launch_gemm_bf16(const GemmArgs& a, bool swap, int bn, int token_tiles, cudaStream_t st) {
+  dim3 grid(a.seg_tile_begin[a.n_seg], token_tiles);
+  if (grid.x == 0 || grid.y == 0) return cudaSuccess;
+  if (swap) {
+    switch (bn) {
+      case 16: return launch_one<16, true>(a, grid, st);
+      case 32: return launch_one<32, true>(a, grid, st);
+      case 64: return launch_one<64, true>(a, grid, st);
+      case 128: return launch_one<128, true>(a, grid, st);
+      case 256: return launch_one<256, true>(a, grid, st);
+    }
+  } else {
+    switch (bn) {
+      case 128: return launch_one<128, false>(a, grid, st);
+      case 256: return launch_one<256, false>(a, grid, st);
+    }
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace gmla

@@ -1,0 +1,616 @@
+// gmla.cu — the C ABI declared in include/gmla.h: argument checks, workspace
+// layout, tensor-map construction and kernel dispatch. Every compute step runs
+// in the kernels of gemm_tc.cu, decode_tc.cu, prefill_tc.cu (bf16, tcgen05) or
+// simt_f32.cu (fp32, CUDA cores); there is no host fallback.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "../../include/gmla.h"
+#include "common.cuh"
+#include "internal.h"
+#include "ptx.cuh"
+
+using namespace gmla;
+
+namespace {
+
+thread_local std::string g_err;
+
+gmla_status fail(gmla_status s, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+gmla_status fail(gmla_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return s;
+}
+
+gmla_status cuda_fail(cudaError_t e, const char* where) {
+  return fail(GMLA_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int num_sms() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// ---------------------------------------------------------------------------
+// tensor maps through the driver entry point (the library does not link libcuda)
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+const char* status_str(gmla_status s) {
+  switch (s) {
+    case GMLA_OK: return "ok";
+    case GMLA_ERR_INVALID_ARG: return "invalid argument";
+    case GMLA_ERR_UNSUPPORTED: return "unsupported shape or mode (no fallback path exists)";
+    case GMLA_ERR_WORKSPACE: return "workspace missing or too small";
+    case GMLA_ERR_CUDA: return "CUDA error";
+    case GMLA_ERR_TIMEOUT: return "a device-side wait timed out";
+    case GMLA_ERR_DEVICE_RANGE: return "a kernel saw an out-of-range sequence length or page";
+  }
+  return "unknown status";
+}
+
+gmla_status check_cfg(const gmla_config* c) {
+  if (!c) return fail(GMLA_ERR_INVALID_ARG, "config is NULL");
+  if (c->d_model <= 0 || c->n_heads <= 0 || c->d_h <= 0 || c->d_c <= 0 || c->d_rope < 0)
+    return fail(GMLA_ERR_INVALID_ARG, "non-positive dimension in config");
+  if (c->d_rope % 2) return fail(GMLA_ERR_INVALID_ARG, "d_rope must be even (RoPE rotates pairs)");
+  if (c->gate_mode != GMLA_GATE_CHANNEL && c->gate_mode != GMLA_GATE_HEAD)
+    return fail(GMLA_ERR_INVALID_ARG, "gate_mode must be GMLA_GATE_CHANNEL or GMLA_GATE_HEAD");
+  if (c->dtype != GMLA_BF16 && c->dtype != GMLA_FP32) return fail(GMLA_ERR_INVALID_ARG, "dtype");
+  if (!(c->softmax_scale > 0.f) || !std::isfinite(c->softmax_scale))
+    return fail(GMLA_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
+  if (c->d_rope && !(c->rope_base > 1.f)) return fail(GMLA_ERR_INVALID_ARG, "rope_base must be > 1");
+  return GMLA_OK;
+}
+
+gmla_status check_ptr(const void* p, const char* name, bool required = true) {
+  if (!p) return required ? fail(GMLA_ERR_INVALID_ARG, "%s is NULL", name) : GMLA_OK;
+  if (!aligned16(p)) return fail(GMLA_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+  return GMLA_OK;
+}
+
+#define GMLA_TRY(x)                         \
+  do {                                      \
+    gmla_status _s = (x);                   \
+    if (_s != GMLA_OK) return _s;           \
+  } while (0)
+
+gmla_status check_cache(const gmla_config* c, const gmla_cache* k) {
+  if (!k) return fail(GMLA_ERR_INVALID_ARG, "cache is NULL");
+  GMLA_TRY(check_ptr(k->data, "cache.data"));
+  if (k->batch <= 0) return fail(GMLA_ERR_INVALID_ARG, "cache.batch must be > 0");
+  if (!k->paged) {
+    if (k->capacity <= 0) return fail(GMLA_ERR_INVALID_ARG, "cache.capacity must be > 0");
+  } else {
+    GMLA_TRY(check_ptr(k->block_table, "cache.block_table"));
+    if (k->page_size <= 0 || k->num_pages <= 0 || k->max_pages_per_seq <= 0)
+      return fail(GMLA_ERR_INVALID_ARG, "paged cache sizes must be > 0");
+    const int ps = k->page_size;
+    const bool ok = (ps < 128) ? (ps >= 8 && (128 % ps) == 0) : (ps % 128 == 0);
+    if (!ok) return fail(GMLA_ERR_UNSUPPORTED, "page_size %d: must divide 128 (>= 8) or be a multiple of 128", ps);
+  }
+  (void)c;
+  return GMLA_OK;
+}
+
+CacheView cache_view(const gmla_config* c, const gmla_cache* k) {
+  CacheView v{};
+  v.data = k->data;
+  v.block_table = k->block_table;
+  v.paged = k->paged;
+  v.batch = k->batch;
+  v.capacity = k->capacity;
+  v.page_size = k->page_size;
+  v.num_pages = k->num_pages;
+  v.max_pages_per_seq = k->max_pages_per_seq;
+  v.row = c->d_c + c->d_rope;
+  return v;
+}
+
+int gate_width(const gmla_config* c) {
+  return c->gate_mode == GMLA_GATE_CHANNEL ? c->n_heads * c->d_h : c->n_heads;
+}
+
+EpiSeg plain_seg(void* out, int64_t row_stride, int block, int block_stride, int col_offset, bool f32,
+                 const float* bias, bool rope, bool scatter) {
+  EpiSeg e{};
+  e.out = out;
+  e.bias = bias;
+  e.row_stride = row_stride;
+  e.block = block;
+  e.block_stride = block_stride;
+  e.col_offset = col_offset;
+  e.out_f32 = f32 ? 1 : 0;
+  e.rope = rope ? 1 : 0;
+  e.cache_scatter = scatter ? 1 : 0;
+  return e;
+}
+
+}  // namespace
+
+namespace gmla {
+
+bool make_tmap_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t row_stride_bytes,
+                  uint32_t box_inner, uint32_t box_rows, bool swizzle128) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {row_stride_bytes};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE,
+            swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_tmap_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t d1, uint64_t d2,
+                  uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box_inner, uint32_t box1, uint32_t box2,
+                  bool swizzle128) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {inner, d1, d2};
+  cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
+  cuuint32_t box[3] = {box_inner, box1, box2};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE,
+            swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace gmla
+
+// ===========================================================================
+// C ABI
+// ===========================================================================
+extern "C" {
+
+const char* gmla_status_string(gmla_status s) { return status_str(s); }
+const char* gmla_last_error(void) { return g_err.c_str(); }
+const char* gmla_version(void) { return "gmla 0.1.0 sm_100a"; }
+
+size_t gmla_latent_project_workspace_size(const gmla_config* cfg, int32_t T) {
+  (void)cfg;
+  (void)T;
+  return 256;
+}
+
+size_t gmla_gate_out_workspace_size(const gmla_config* cfg, int32_t T) {
+  if (!cfg || T < 0) return 256;
+  const size_t es = cfg->dtype == GMLA_FP32 ? 4 : 2;
+  return 256 + align256(static_cast<size_t>(T) * cfg->n_heads * cfg->d_h * es);
+}
+
+size_t gmla_decode_workspace_size(const gmla_config* cfg, int32_t B) {
+  if (!cfg || B < 0) return 256;
+  if (cfg->dtype == GMLA_FP32) return 256;
+  return decode_layout(B, cfg->n_heads, cfg->d_c, cfg->d_rope, num_sms()).total;
+}
+
+size_t gmla_prefill_workspace_size(const gmla_config* cfg, int32_t T, int32_t B) {
+  if (!cfg || T < 0 || B < 0) return 256;
+  const size_t es = cfg->dtype == GMLA_FP32 ? 4 : 2;
+  const size_t kv = static_cast<size_t>(T) * cfg->n_heads * cfg->d_h * es;
+  return 256 + 2 * align256(kv);
+}
+
+gmla_status gmla_clear_status(void* workspace, void* stream) {
+  if (!workspace) return fail(GMLA_ERR_WORKSPACE, "workspace is NULL");
+  cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(int), static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? GMLA_OK : cuda_fail(e, "gmla_clear_status");
+}
+
+gmla_status gmla_sync_status(const void* workspace, void* stream) {
+  if (!workspace) return fail(GMLA_ERR_WORKSPACE, "workspace is NULL");
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "gmla_sync_status: stream");
+  int v = 0;
+  e = cudaMemcpy(&v, workspace, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "gmla_sync_status: read");
+  if (v == kStatusTimeout) return fail(GMLA_ERR_TIMEOUT, "a device-side wait timed out");
+  if (v == kStatusRange) return fail(GMLA_ERR_DEVICE_RANGE, "a kernel saw an out-of-range length or page");
+  return v == 0 ? GMLA_OK : fail(GMLA_ERR_CUDA, "unknown device status %d", v);
+}
+
+// ---------------------------------------------------------------------------
+gmla_status gmla_latent_project(const gmla_config* cfg, const gmla_weights* w, const void* x, int32_t T,
+                                const int32_t* positions, const int32_t* seq_ids, const gmla_cache* cache,
+                                void* q_out, float* gate_logits, void* workspace, size_t workspace_bytes,
+                                void* stream) {
+  GMLA_TRY(check_cfg(cfg));
+  if (!w) return fail(GMLA_ERR_INVALID_ARG, "weights is NULL");
+  if (T < 0) return fail(GMLA_ERR_INVALID_ARG, "T < 0");
+  GMLA_TRY(check_cache(cfg, cache));
+  if (!workspace || workspace_bytes < gmla_latent_project_workspace_size(cfg, T))
+    return fail(GMLA_ERR_WORKSPACE, "latent_project needs %zu workspace bytes",
+                gmla_latent_project_workspace_size(cfg, T));
+  if (T == 0) return GMLA_OK;
+  GMLA_TRY(check_ptr(x, "x"));
+  GMLA_TRY(check_ptr(positions, "positions"));
+  GMLA_TRY(check_ptr(seq_ids, "seq_ids"));
+  GMLA_TRY(check_ptr(q_out, "q_out"));
+  GMLA_TRY(check_ptr(gate_logits, "gate_logits"));
+  GMLA_TRY(check_ptr(w->W_c, "W_c"));
+  GMLA_TRY(check_ptr(w->W_q, "W_q"));
+  GMLA_TRY(check_ptr(w->W_g, "W_g"));
+  if (cfg->d_rope) {
+    GMLA_TRY(check_ptr(w->W_kr, "W_kr"));
+    GMLA_TRY(check_ptr(w->W_qr, "W_qr"));
+  }
+  if (cfg->gate_bias) GMLA_TRY(check_ptr(w->b_g, "b_g"));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int H = cfg->n_heads, dh = cfg->d_h, dc = cfg->d_c, dr = cfg->d_rope, dm = cfg->d_model;
+  const int row = dc + dr, G = gate_width(cfg);
+  const int dq = dh + dr;
+  const CacheView cv = cache_view(cfg, cache);
+  int* status = static_cast<int*>(workspace);
+
+  // segments of the weight dimension: [W_c | W_kr | W_q | W_qr | W_g]
+  struct Seg {
+    const void* W;
+    int rows;
+    EpiSeg e;
+  } segs[kMaxSeg];
+  int ns = 0;
+  const bool f32 = cfg->dtype == GMLA_FP32;
+  segs[ns++] = {w->W_c, dc, plain_seg(cache->data, row, 1 << 30, 0, 0, f32, nullptr, false, true)};
+  if (dr) segs[ns++] = {w->W_kr, dr, plain_seg(cache->data, row, dr, 0, dc, f32, nullptr, true, true)};
+  segs[ns++] = {w->W_q, H * dh, plain_seg(q_out, static_cast<int64_t>(H) * dq, dh, dq, 0, f32, nullptr, false, false)};
+  if (dr)
+    segs[ns++] = {w->W_qr, H * dr, plain_seg(q_out, static_cast<int64_t>(H) * dq, dr, dq, dh, f32, nullptr, true, false)};
+  segs[ns++] = {w->W_g, G,
+                plain_seg(gate_logits, G, 1 << 30, 0, 0, true, cfg->gate_bias ? w->b_g : nullptr, false, false)};
+
+  if (f32) {
+    F32Args a{};
+    a.x = static_cast<const float*>(x);
+    a.T = T;
+    a.K = dm;
+    a.n_seg = ns;
+    for (int i = 0; i < ns; ++i) {
+      a.W[i] = static_cast<const float*>(segs[i].W);
+      a.epi[i] = segs[i].e;
+      a.seg_rows[i] = segs[i].rows;
+    }
+    a.positions = positions;
+    a.seq_ids = seq_ids;
+    a.cache = cv;
+    a.log2_rope_base = dr ? std::log2(static_cast<double>(cfg->rope_base)) : 0.0;
+    a.status = status;
+    cudaError_t e = launch_gemm_f32(a, st);
+    return e == cudaSuccess ? GMLA_OK : cuda_fail(e, "latent_project (fp32)");
+  }
+
+  if (dm % 8) return fail(GMLA_ERR_UNSUPPORTED, "bf16 path needs d_model %% 8 == 0");
+  GemmArgs a{};
+  const bool swap = T <= 256;
+  const int bn = swap ? (T <= 16 ? 16 : T <= 32 ? 32 : T <= 64 ? 64 : T <= 128 ? 128 : 256) : 256;
+  const int wtile = gemm_weight_tile(swap, bn);
+  if (!make_tmap_2d(&a.act, x, dm, T, static_cast<uint64_t>(dm) * 2, 64, swap ? bn : 128, true))
+    return fail(GMLA_ERR_CUDA, "tensor map for x failed");
+  a.seg_tile_begin[0] = 0;
+  for (int i = 0; i < ns; ++i) {
+    if (!make_tmap_2d(&a.wt[i], segs[i].W, dm, segs[i].rows, static_cast<uint64_t>(dm) * 2, 64, wtile, true))
+      return fail(GMLA_ERR_CUDA, "tensor map for weight segment %d failed", i);
+    a.epi[i] = segs[i].e;
+    a.seg_rows[i] = segs[i].rows;
+    a.seg_tile_begin[i + 1] = a.seg_tile_begin[i] + (segs[i].rows + wtile - 1) / wtile;
+  }
+  a.n_seg = ns;
+  a.T = T;
+  a.K = dm;
+  a.row_mode = 0;
+  a.positions = positions;
+  a.seq_ids = seq_ids;
+  a.cache = cv;
+  a.log2_rope_base = dr ? std::log2(static_cast<double>(cfg->rope_base)) : 0.0;
+  a.status = status;
+  const int ttiles = swap ? (T + bn - 1) / bn : (T + 127) / 128;
+  cudaError_t e = launch_gemm_bf16(a, swap, bn, ttiles, st);
+  return e == cudaSuccess ? GMLA_OK : cuda_fail(e, "latent_project");
+}
+
+// ---------------------------------------------------------------------------
+gmla_status gmla_decode(const gmla_config* cfg, const gmla_weights* w, const void* q, const float* gate_logits,
+                        const gmla_cache* cache, const int32_t* seq_lens, int32_t B, void* o_gated,
+                        void* workspace, size_t workspace_bytes, void* stream) {
+  GMLA_TRY(check_cfg(cfg));
+  if (!w) return fail(GMLA_ERR_INVALID_ARG, "weights is NULL");
+  if (B < 0) return fail(GMLA_ERR_INVALID_ARG, "B < 0");
+  GMLA_TRY(check_cache(cfg, cache));
+  const size_t need = gmla_decode_workspace_size(cfg, B);
+  if (!workspace || workspace_bytes < need)
+    return fail(GMLA_ERR_WORKSPACE, "decode needs %zu workspace bytes, got %zu", need, workspace_bytes);
+  GMLA_TRY(check_ptr(workspace, "workspace"));
+  if (B == 0) return GMLA_OK;
+  if (B > cache->batch) return fail(GMLA_ERR_INVALID_ARG, "B (%d) exceeds cache.batch (%d)", B, cache->batch);
+  GMLA_TRY(check_ptr(q, "q"));
+  GMLA_TRY(check_ptr(seq_lens, "seq_lens"));
+  GMLA_TRY(check_ptr(o_gated, "o_gated"));
+  GMLA_TRY(check_ptr(gate_logits, "gate_logits", false));
+  GMLA_TRY(check_ptr(w->W_k, "W_k"));
+  GMLA_TRY(check_ptr(w->W_v, "W_v"));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const CacheView cv = cache_view(cfg, cache);
+  int* status = static_cast<int*>(workspace);
+
+  if (cfg->dtype == GMLA_FP32) {
+    AttnF32Args a{};
+    a.q = static_cast<const float*>(q);
+    a.cache = static_cast<const float*>(cache->data);
+    a.cv = cv;
+    a.W_k = static_cast<const float*>(w->W_k);
+    a.W_v = static_cast<const float*>(w->W_v);
+    a.gate_logits = gate_logits;
+    a.o = static_cast<float*>(o_gated);
+    a.cu_seqlens = nullptr;
+    a.seq_lens = seq_lens;
+    a.B = B;
+    a.T = B;
+    a.H = cfg->n_heads;
+    a.d_h = cfg->d_h;
+    a.d_c = cfg->d_c;
+    a.d_rope = cfg->d_rope;
+    a.gate_mode = cfg->gate_mode;
+    a.scale = cfg->softmax_scale;
+    a.status = status;
+    cudaError_t e = launch_attn_f32(a, st);
+    return e == cudaSuccess ? GMLA_OK : cuda_fail(e, "decode (fp32)");
+  }
+
+  if (cfg->d_c != 512 || (cfg->d_rope != 0 && cfg->d_rope != 64))
+    return fail(GMLA_ERR_UNSUPPORTED, "bf16 decode covers d_c = 512 with d_rope in {0, 64}");
+  if (cfg->d_h % 4 || cfg->d_h > 256) return fail(GMLA_ERR_UNSUPPORTED, "bf16 decode needs d_h %% 4 == 0, <= 256");
+  const DecodeLayout L = decode_layout(B, cfg->n_heads, cfg->d_c, cfg->d_rope, num_sms());
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  DecodeArgs a{};
+  const int row = cfg->d_c + cfg->d_rope;
+  if (!cache->paged) {
+    if (!make_tmap_2d(&a.cache_map, cache->data, row, static_cast<uint64_t>(cache->batch) * cache->capacity,
+                      static_cast<uint64_t>(row) * 2, 64, 128, true))
+      return fail(GMLA_ERR_CUDA, "tensor map for the cache failed");
+  } else {
+    const int ps = cache->page_size;
+    if (!make_tmap_3d(&a.cache_map, cache->data, row, ps, cache->num_pages, static_cast<uint64_t>(row) * 2,
+                      static_cast<uint64_t>(row) * 2 * ps, 64, ps < 128 ? ps : 128, 1, true))
+      return fail(GMLA_ERR_CUDA, "tensor map for the paged cache failed");
+  }
+  if (!make_tmap_2d(&a.qa_map, ws + L.off_qa, row, static_cast<uint64_t>(B) * cfg->n_heads,
+                    static_cast<uint64_t>(row) * 2, 64, L.HG, true))
+    return fail(GMLA_ERR_CUDA, "tensor map for the absorbed queries failed");
+  a.cache = cv;
+  a.seq_lens = seq_lens;
+  a.q = q;
+  a.W_k = w->W_k;
+  a.W_v = w->W_v;
+  a.gate_logits = gate_logits;
+  a.o = o_gated;
+  a.qa = ws + L.off_qa;
+  a.o_part = reinterpret_cast<float*>(ws + L.off_opart);
+  a.ml_part = reinterpret_cast<float*>(ws + L.off_ml);
+  a.seg_info = reinterpret_cast<int4*>(ws + L.off_seg);
+  a.seq_first_seg = reinterpret_cast<int32_t*>(ws + L.off_seqfirst);
+  a.cta_first_seg = reinterpret_cast<int32_t*>(ws + L.off_ctafirst);
+  a.status = status;
+  a.B = B;
+  a.H = cfg->n_heads;
+  a.d_h = cfg->d_h;
+  a.d_c = cfg->d_c;
+  a.d_rope = cfg->d_rope;
+  a.gate_mode = cfg->gate_mode;
+  a.HG = L.HG;
+  a.n_hg = L.n_hg;
+  a.G = L.G;
+  a.max_seg = L.max_seg;
+  a.q_scale = cfg->softmax_scale * 1.4426950408889634f;
+  cudaError_t e = launch_decode_bf16(a, st);
+  return e == cudaSuccess ? GMLA_OK : cuda_fail(e, "decode");
+}
+
+// ---------------------------------------------------------------------------
+gmla_status gmla_prefill(const gmla_config* cfg, const gmla_weights* w, const void* q, const float* gate_logits,
+                         const gmla_cache* cache, const int32_t* cu_seqlens, int32_t B, int32_t T,
+                         int32_t max_seqlen, void* o_gated, void* workspace, size_t workspace_bytes,
+                         void* stream) {
+  GMLA_TRY(check_cfg(cfg));
+  if (!w) return fail(GMLA_ERR_INVALID_ARG, "weights is NULL");
+  if (B < 0 || T < 0 || max_seqlen < 0) return fail(GMLA_ERR_INVALID_ARG, "negative size");
+  GMLA_TRY(check_cache(cfg, cache));
+  const size_t need = gmla_prefill_workspace_size(cfg, T, B);
+  if (!workspace || workspace_bytes < need)
+    return fail(GMLA_ERR_WORKSPACE, "prefill needs %zu workspace bytes, got %zu", need, workspace_bytes);
+  GMLA_TRY(check_ptr(workspace, "workspace"));
+  if (B == 0 || T == 0) return GMLA_OK;
+  if (B > cache->batch) return fail(GMLA_ERR_INVALID_ARG, "B (%d) exceeds cache.batch (%d)", B, cache->batch);
+  if (cache->paged) return fail(GMLA_ERR_UNSUPPORTED, "prefill reads a contiguous cache");
+  if (max_seqlen > cache->capacity) return fail(GMLA_ERR_INVALID_ARG, "max_seqlen exceeds cache.capacity");
+  GMLA_TRY(check_ptr(q, "q"));
+  GMLA_TRY(check_ptr(cu_seqlens, "cu_seqlens"));
+  GMLA_TRY(check_ptr(o_gated, "o_gated"));
+  GMLA_TRY(check_ptr(gate_logits, "gate_logits", false));
+  GMLA_TRY(check_ptr(w->W_k, "W_k"));
+  GMLA_TRY(check_ptr(w->W_v, "W_v"));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int* status = static_cast<int*>(workspace);
+  const CacheView cv = cache_view(cfg, cache);
+
+  if (cfg->dtype == GMLA_FP32) {
+    AttnF32Args a{};
+    a.q = static_cast<const float*>(q);
+    a.cache = static_cast<const float*>(cache->data);
+    a.cv = cv;
+    a.W_k = static_cast<const float*>(w->W_k);
+    a.W_v = static_cast<const float*>(w->W_v);
+    a.gate_logits = gate_logits;
+    a.o = static_cast<float*>(o_gated);
+    a.cu_seqlens = cu_seqlens;
+    a.seq_lens = nullptr;
+    a.B = B;
+    a.T = T;
+    a.H = cfg->n_heads;
+    a.d_h = cfg->d_h;
+    a.d_c = cfg->d_c;
+    a.d_rope = cfg->d_rope;
+    a.gate_mode = cfg->gate_mode;
+    a.max_len = max_seqlen;
+    a.scale = cfg->softmax_scale;
+    a.status = status;
+    cudaError_t e = launch_attn_f32(a, st);
+    return e == cudaSuccess ? GMLA_OK : cuda_fail(e, "prefill (fp32)");
+  }
+
+  if (cfg->d_rope != 0) return fail(GMLA_ERR_UNSUPPORTED, "bf16 prefill covers NoPE (d_rope = 0)");
+  if (cfg->d_h != 128) return fail(GMLA_ERR_UNSUPPORTED, "bf16 prefill covers d_h = 128");
+  if (cfg->d_c % 64) return fail(GMLA_ERR_UNSUPPORTED, "bf16 prefill needs d_c %% 64 == 0");
+  const int H = cfg->n_heads, HD = H * cfg->d_h;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const size_t kv_bytes = align256(static_cast<size_t>(T) * HD * 2);
+  void* Kbuf = ws + 256;
+  void* Vbuf = ws + 256 + kv_bytes;
+
+  // K^(h), V^(h) = C W_k^(h)T, C W_v^(h)T for every prompt token
+  GemmArgs g{};
+  const int bn = 256;
+  const int tps = (max_seqlen + 127) / 128;
+  if (!make_tmap_2d(&g.act, cache->data, cfg->d_c, static_cast<uint64_t>(cache->batch) * cache->capacity,
+                    static_cast<uint64_t>(cv.row) * 2, 64, 128, true))
+    return fail(GMLA_ERR_CUDA, "tensor map for cache latents failed");
+  const void* Ws[2] = {w->W_k, w->W_v};
+  void* outs[2] = {Kbuf, Vbuf};
+  g.seg_tile_begin[0] = 0;
+  for (int i = 0; i < 2; ++i) {
+    if (!make_tmap_2d(&g.wt[i], Ws[i], cfg->d_c, HD, static_cast<uint64_t>(cfg->d_c) * 2, 64, bn, true))
+      return fail(GMLA_ERR_CUDA, "tensor map for W_k/W_v failed");
+    g.epi[i] = plain_seg(outs[i], HD, 1 << 30, 0, 0, false, nullptr, false, false);
+    g.seg_rows[i] = HD;
+    g.seg_tile_begin[i + 1] = g.seg_tile_begin[i] + (HD + bn - 1) / bn;
+  }
+  g.n_seg = 2;
+  g.T = T;
+  g.K = cfg->d_c;
+  g.row_mode = 1;
+  g.tiles_per_seq = tps;
+  g.act_seq_stride = cache->capacity;
+  g.cu_seqlens = cu_seqlens;
+  g.status = status;
+  cudaError_t e = launch_gemm_bf16(g, false, bn, B * tps, st);
+  if (e != cudaSuccess) return cuda_fail(e, "prefill K/V rebuild");
+
+  PrefillArgs p{};
+  const int dq = cfg->d_h + cfg->d_rope;
+  if (!make_tmap_2d(&p.q_map, q, static_cast<uint64_t>(H) * dq, T, static_cast<uint64_t>(H) * dq * 2, 64, 128, true) ||
+      !make_tmap_2d(&p.k_map, Kbuf, HD, T, static_cast<uint64_t>(HD) * 2, 64, 128, true) ||
+      !make_tmap_2d(&p.v_map, Vbuf, HD, T, static_cast<uint64_t>(HD) * 2, 64, 128, true))
+    return fail(GMLA_ERR_CUDA, "tensor maps for prefill attention failed");
+  p.gate_logits = gate_logits;
+  p.o = o_gated;
+  p.cu_seqlens = cu_seqlens;
+  p.status = status;
+  p.B = B;
+  p.T = T;
+  p.H = H;
+  p.d_h = cfg->d_h;
+  p.gate_mode = cfg->gate_mode;
+  p.q_tiles_per_seq = tps;
+  p.scale_log2 = cfg->softmax_scale * 1.4426950408889634f;
+  e = launch_prefill_attn_bf16(p, st);
+  return e == cudaSuccess ? GMLA_OK : cuda_fail(e, "prefill attention");
+}
+
+// ---------------------------------------------------------------------------
+gmla_status gmla_gate_out(const gmla_config* cfg, const gmla_weights* w, const void* o, int32_t T,
+                          const float* gate_logits, void* y, void* workspace, size_t workspace_bytes,
+                          void* stream) {
+  GMLA_TRY(check_cfg(cfg));
+  if (!w) return fail(GMLA_ERR_INVALID_ARG, "weights is NULL");
+  if (T < 0) return fail(GMLA_ERR_INVALID_ARG, "T < 0");
+  const size_t need = gmla_gate_out_workspace_size(cfg, T);
+  if (!workspace || workspace_bytes < need)
+    return fail(GMLA_ERR_WORKSPACE, "gate_out needs %zu workspace bytes, got %zu", need, workspace_bytes);
+  GMLA_TRY(check_ptr(workspace, "workspace"));
+  if (T == 0) return GMLA_OK;
+  GMLA_TRY(check_ptr(o, "o"));
+  GMLA_TRY(check_ptr(y, "y"));
+  GMLA_TRY(check_ptr(w->W_o, "W_o"));
+  GMLA_TRY(check_ptr(gate_logits, "gate_logits", false));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int HD = cfg->n_heads * cfg->d_h, dm = cfg->d_model;
+  const bool f32 = cfg->dtype == GMLA_FP32;
+  int* status = static_cast<int*>(workspace);
+  const void* src = o;
+  if (gate_logits) {
+    void* tmp = static_cast<uint8_t*>(workspace) + 256;
+    cudaError_t e = launch_gate_apply(o, gate_logits, tmp, T, cfg->n_heads, cfg->d_h, cfg->gate_mode, f32, st);
+    if (e != cudaSuccess) return cuda_fail(e, "gate_out: gate");
+    src = tmp;
+  }
+  const EpiSeg ep = plain_seg(y, dm, 1 << 30, 0, 0, f32, nullptr, false, false);
+  if (f32) {
+    F32Args a{};
+    a.x = static_cast<const float*>(src);
+    a.T = T;
+    a.K = HD;
+    a.W[0] = static_cast<const float*>(w->W_o);
+    a.epi[0] = ep;
+    a.seg_rows[0] = dm;
+    a.n_seg = 1;
+    a.status = status;
+    cudaError_t e = launch_gemm_f32(a, st);
+    return e == cudaSuccess ? GMLA_OK : cuda_fail(e, "gate_out (fp32)");
+  }
+  if (HD % 8) return fail(GMLA_ERR_UNSUPPORTED, "bf16 path needs H*d_h %% 8 == 0");
+  GemmArgs a{};
+  const bool swap = T <= 256;
+  const int bn = swap ? (T <= 16 ? 16 : T <= 32 ? 32 : T <= 64 ? 64 : T <= 128 ? 128 : 256) : 256;
+  const int wtile = gemm_weight_tile(swap, bn);
+  if (!make_tmap_2d(&a.act, src, HD, T, static_cast<uint64_t>(HD) * 2, 64, swap ? bn : 128, true) ||
+      !make_tmap_2d(&a.wt[0], w->W_o, HD, dm, static_cast<uint64_t>(HD) * 2, 64, wtile, true))
+    return fail(GMLA_ERR_CUDA, "tensor maps for gate_out failed");
+  a.epi[0] = ep;
+  a.seg_rows[0] = dm;
+  a.seg_tile_begin[0] = 0;
+  a.seg_tile_begin[1] = (dm + wtile - 1) / wtile;
+  a.n_seg = 1;
+  a.T = T;
+  a.K = HD;
+  a.row_mode = 0;
+  a.status = status;
+  const int ttiles = swap ? (T + bn - 1) / bn : (T + 127) / 128;
+  cudaError_t e = launch_gemm_bf16(a, swap, bn, ttiles, st);
+  return e == cudaSuccess ? GMLA_OK : cuda_fail(e, "gate_out");
+}
+
+}  // extern "C"

@@ -1,0 +1,105 @@
+// internal.h — declarations shared between the C-ABI layer and the kernels.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace gmla {
+
+// ----- tcgen05 GEMM (gemm_tc.cu) -----
+cudaError_t launch_gemm_bf16(const GemmArgs& a, bool swap, int bn, int token_tiles, cudaStream_t st);
+int gemm_weight_tile(bool swap, int bn);
+
+// ----- decode (decode_tc.cu) -----
+struct DecodeArgs {
+  CUtensorMap cache_map;     // contiguous: 2D [B*cap, row]; paged: 3D [pages, page_size, row]
+  CUtensorMap qa_map;        // 2D [B*H, row] bf16 absorbed queries
+  CacheView cache;
+  const int32_t* seq_lens;   // [B]
+  const void* q;             // [B, H, d_h + d_R]
+  const void* W_k;           // [H, d_h, d_c]
+  const void* W_v;           // [H, d_h, d_c]
+  const float* gate_logits;  // [B, G] or null
+  void* o;                   // [B, H*d_h]
+  void* qa;                  // workspace: [B*H, row] bf16
+  float* o_part;             // workspace: [n_hg, max_seg, HG, d_c]
+  float* ml_part;            // workspace: [n_hg, max_seg, HG, 2]
+  int4* seg_info;            // workspace: [max_seg]
+  int32_t* seq_first_seg;    // workspace: [B + 1]
+  int32_t* cta_first_seg;    // workspace: [G + 1]
+  int* status;
+  int32_t B, H, d_h, d_c, d_rope, gate_mode;
+  int32_t HG, n_hg, G, max_seg;
+  float q_scale;             // softmax_scale * log2(e), folded into the absorbed query
+};
+
+struct DecodeLayout {
+  size_t off_qa, off_opart, off_ml, off_seg, off_seqfirst, off_ctafirst, total;
+  int HG, n_hg, G, max_seg;
+};
+DecodeLayout decode_layout(int B, int H, int d_c, int d_rope, int num_sms);
+cudaError_t launch_decode_bf16(DecodeArgs& a, cudaStream_t st);
+
+// ----- fp32 CUDA-core path (simt_f32.cu) -----
+struct F32Args {
+  const float* x;            // [T, K] activations
+  int32_t T, K;
+  const float* W[kMaxSeg];   // segment weights [rows, K]
+  EpiSeg epi[kMaxSeg];
+  int32_t seg_rows[kMaxSeg];
+  int32_t seg_tile_begin[kMaxSeg + 1];   // filled by launch_gemm_f32
+  int32_t n_seg;
+  const int32_t* positions;
+  const int32_t* seq_ids;
+  CacheView cache;
+  double log2_rope_base;
+  int* status;
+};
+cudaError_t launch_gemm_f32(F32Args a, cudaStream_t st);
+
+struct AttnF32Args {
+  const float* q;            // [T or B, H, d_h + d_R]
+  const float* cache;        // cache rows (fp32)
+  CacheView cv;
+  const float* W_k;
+  const float* W_v;
+  const float* gate_logits;
+  float* o;
+  const int32_t* cu_seqlens; // prefill: [B+1]; null for decode
+  const int32_t* seq_lens;   // decode: [B]
+  int32_t B, T, H, d_h, d_c, d_rope, gate_mode, max_len;
+  float scale;
+  float* scratch;            // [B*H*(d_c + max_len)] or per-launch scratch
+  int* status;
+};
+cudaError_t launch_attn_f32(const AttnF32Args& a, cudaStream_t st);
+
+// ----- prefill (prefill_tc.cu) -----
+struct PrefillArgs {
+  CUtensorMap q_map;         // 2D [T, H*(d_h+d_R)] bf16
+  CUtensorMap k_map;         // 2D [T, H*d_h] bf16
+  CUtensorMap v_map;         // 2D [T, H*d_h] bf16
+  const float* gate_logits;  // [T, G] or null
+  void* o;                   // [T, H*d_h]
+  const int32_t* cu_seqlens;
+  int* status;
+  int32_t B, T, H, d_h, gate_mode, q_tiles_per_seq;
+  float scale_log2;
+};
+cudaError_t launch_prefill_attn_bf16(const PrefillArgs& a, cudaStream_t st);
+
+// ----- elementwise helpers (gmla.cu) -----
+cudaError_t launch_gate_apply(const void* o, const float* g, void* out, int T, int H, int d_h, int gate_mode,
+                              int is_f32, cudaStream_t st);
+
+// ----- tensor maps -----
+bool make_tmap_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t row_stride_bytes,
+                  uint32_t box_inner, uint32_t box_rows, bool swizzle128);
+bool make_tmap_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t d1, uint64_t d2,
+                  uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box_inner, uint32_t box1,
+                  uint32_t box2, bool swizzle128);
+
+}  // namespace gmla

@@ -1,0 +1,220 @@
+/*
+ * gmla.h — C ABI of the Gated Multi-head Latent Attention hot path (B200, sm_100a).
+ *
+ * What is computed (sources cited by page title and section):
+ *
+ *   "Gated MLA 计算公式：输出门与 FFN 的区别" (hackcha.cn)
+ *     §一   c_s = W_c x_s;  k_s^(h) = W_k^(h) c_s;  v_s^(h) = W_v^(h) c_s
+ *     §二   a_{t,s} = Softmax_{s<=t}(q_t^(h) . k_s^(h) / sqrt(d_h)),  o_t^(h) = sum_s a_{t,s} v_s^(h)
+ *           õ_t = Concat_h o_t^(h);   y_t = W_o [ Sigmoid(W_g x_t) ⊙ õ_t ]   (boxed equation)
+ *     §四   NoPE: no positional encoding on q and k.
+ *   "Gated Multi-head Latent Attention (Gated MLA)" (codewithdark-git.github.io)
+ *     "Gating Mechanism": per-head gate g_h = sigmoid(W_g x + b_g) scaling head h.
+ *   "LLM 注意力与计算内核精读笔记 · 03 注意力头变体：MQA / GQA / MLA" (zzszmyf.github.io)
+ *     §5.1  only c_s is cached; W_k and W_v are absorbed at inference time.
+ *     §5.2  decoupled RoPE: k^R_s = RoPE(W_kr x_s) is cached beside c_s, shared by
+ *           all heads; q^R gets its own rotated d_R dims per head.
+ *     §5.3  a cached row holds d_c + d_R elements (576 for d_c=512, d_R=64).
+ *     题4   absorption identity q^T W_k c = (W_k^T q)^T c.
+ *
+ * Readings where the pages leave a step open (shared with the oracle):
+ *   q^(h) = W_q^(h) x (full-rank query, no bias); softmax_scale is passed in
+ *   (1/sqrt(d_h), or 1/sqrt(d_h + d_R) with the decoupled RoPE key); RoPE rotates
+ *   pairs (2i, 2i+1) by pos * base^(-2i/d_R); a decode query is at position
+ *   seq_len - 1 and attends to all seq_len cached rows.
+ *
+ * Conventions for every entry point:
+ *   - Every pointer argument is a DEVICE pointer owned by the caller unless its
+ *     comment says otherwise; the library keeps none of them after the call.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream). The returned status covers argument checks and the
+ *     launches. Faults seen by a kernel (a device wait that timed out, a
+ *     sequence longer than its cache) are written to a status word at the start
+ *     of `workspace` and returned by gmla_sync_status().
+ *   - Row-major layouts. Weights are [out, in]:
+ *       W_c [d_c, d_model]   W_kr [d_R, d_model]    W_q [H*d_h, d_model]
+ *       W_qr [H*d_R, d_model]  W_k, W_v [H, d_h, d_c]
+ *       W_g [G, d_model] with G = H*d_h (per-channel gate) or G = H (per-head gate)
+ *       b_g [G] (fp32, optional)   W_o [d_model, H*d_h]
+ *     Weights, x, q, the cache, o and y use the config's dtype (bf16 or fp32);
+ *     gate logits and b_g are always fp32; index arrays are int32.
+ *   - The bf16 path runs on tcgen05 tensor cores with fp32 accumulation; the
+ *     fp32 path runs on CUDA cores in fp32. There is no CPU fallback: a shape
+ *     the kernels do not cover returns GMLA_ERR_UNSUPPORTED.
+ *   - All base pointers must be 16-byte aligned.
+ */
+#ifndef GMLA_H_
+#define GMLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define GMLA_API __attribute__((visibility("default")))
+#else
+#define GMLA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum gmla_status {
+  GMLA_OK = 0,
+  GMLA_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, inconsistent sizes */
+  GMLA_ERR_UNSUPPORTED = 2,   /* valid but not covered by the kernels (no fallback) */
+  GMLA_ERR_WORKSPACE = 3,     /* workspace missing or smaller than the *_workspace_size query */
+  GMLA_ERR_CUDA = 4,          /* a CUDA runtime/driver call failed; see gmla_last_error() */
+  GMLA_ERR_TIMEOUT = 5,       /* a device-side wait gave up (reported by gmla_sync_status) */
+  GMLA_ERR_DEVICE_RANGE = 6   /* a kernel saw an out-of-range length/page (gmla_sync_status) */
+} gmla_status;
+
+typedef enum gmla_dtype { GMLA_BF16 = 0, GMLA_FP32 = 1 } gmla_dtype;
+
+/* Per-channel gate: G = H*d_h ("Gated MLA 计算公式" §二 boxed equation).
+ * Per-head gate:    G = H, broadcast over the head's d_h channels
+ *                   ("Gated Multi-head Latent Attention", "Gating Mechanism"). */
+typedef enum gmla_gate_mode { GMLA_GATE_CHANNEL = 0, GMLA_GATE_HEAD = 1 } gmla_gate_mode;
+
+typedef struct gmla_config {
+  int32_t d_model;
+  int32_t n_heads;        /* H */
+  int32_t d_h;            /* head dim of q, k, v */
+  int32_t d_c;            /* latent dim (cached) */
+  int32_t d_rope;         /* decoupled RoPE dims d_R; 0 = NoPE */
+  int32_t gate_mode;      /* gmla_gate_mode */
+  int32_t gate_bias;      /* 1: b_g is given */
+  float softmax_scale;    /* scale applied to q.k (+ q^R.k^R) before the softmax */
+  float rope_base;        /* RoPE base (e.g. 10000) */
+  int32_t dtype;          /* gmla_dtype */
+} gmla_config;
+
+typedef struct gmla_weights {
+  const void* W_c;
+  const void* W_kr;       /* NULL when d_rope == 0 */
+  const void* W_q;
+  const void* W_qr;       /* NULL when d_rope == 0 */
+  const void* W_k;
+  const void* W_v;
+  const void* W_g;
+  const float* b_g;       /* NULL unless gate_bias */
+  const void* W_o;
+} gmla_weights;
+
+/* Latent cache. A row holds [c (d_c) | k^R (d_R)] of one token, d_c + d_R
+ * elements ("精读笔记 03" §5.2). Nothing gate-related is cached: the gate
+ * depends only on the current token ("Gated MLA 计算公式" §五).
+ *   contiguous (paged = 0): data = [batch, capacity, d_c + d_R]
+ *   paged      (paged = 1): data = [num_pages, page_size, d_c + d_R];
+ *     token p of sequence b lives in page block_table[b*max_pages_per_seq + p/page_size]
+ *     at row p % page_size. block_table is a device int32 array. */
+typedef struct gmla_cache {
+  void* data;
+  int32_t paged;
+  int32_t batch;              /* contiguous: sequences held */
+  int32_t capacity;           /* contiguous: rows per sequence */
+  int32_t page_size;          /* paged: rows per page (multiple of 8) */
+  int32_t num_pages;          /* paged: pages in the pool */
+  int32_t max_pages_per_seq;  /* paged: row length of block_table */
+  const int32_t* block_table; /* paged: [batch, max_pages_per_seq] */
+} gmla_cache;
+
+/* ---------------------------------------------------------------------------
+ * gmla_latent_project — everything computed from the tokens' own hidden states.
+ *   x            [T, d_model]
+ *   positions    [T] int32, position of each token within its sequence
+ *   seq_ids      [T] int32, sequence (cache slot) of each token
+ *   cache        receives row [c | RoPE(W_kr x, pos)] of every token at (seq_id, position)
+ *                ("Gated MLA 计算公式" §一; "精读笔记 03" §5.1, §5.2)
+ *   q_out        [T, H, d_h + d_R]: q^(h) = W_q^(h) x, then q^R = RoPE(W_qr^(h) x, pos)
+ *   gate_logits  [T, G] fp32: W_g x (+ b_g)
+ *   workspace    device scratch of gmla_latent_project_workspace_size(cfg, T) bytes
+ * Rows of the cache not addressed by (seq_id, position) are left untouched.
+ * Returns GMLA_ERR_INVALID_ARG if T < 0 or a pointer is missing/misaligned.
+ * ------------------------------------------------------------------------- */
+GMLA_API gmla_status gmla_latent_project(const gmla_config* cfg, const gmla_weights* w,
+                                const void* x, int32_t T,
+                                const int32_t* positions, const int32_t* seq_ids,
+                                const gmla_cache* cache,
+                                void* q_out, float* gate_logits,
+                                void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * gmla_decode — one query token per sequence against its cached rows, in the
+ * absorbed form ("精读笔记 03" §5.1, 题4): scores are (W_k^T q) . c_s (+ q^R . k^R_s),
+ * the weighted sum is taken over latents and W_v is applied afterwards; the
+ * sigmoid gate is applied before the result leaves the chip.
+ *   q            [B, H, d_h + d_R] (as written by gmla_latent_project)
+ *   gate_logits  [B, G] fp32, or NULL to write the ungated head outputs
+ *   seq_lens     [B] int32: cached rows of each sequence INCLUDING the query's
+ *                own row; the query sits at position seq_len - 1. A length of 0
+ *                yields o = 0; a length beyond the cache sets
+ *                GMLA_ERR_DEVICE_RANGE in the status word and yields o = 0.
+ *   o_gated      [B, H*d_h] = gate ⊙ Concat_h o^(h)
+ *   workspace    device scratch of gmla_decode_workspace_size(cfg, B) bytes
+ * ------------------------------------------------------------------------- */
+GMLA_API gmla_status gmla_decode(const gmla_config* cfg, const gmla_weights* w,
+                        const void* q, const float* gate_logits,
+                        const gmla_cache* cache, const int32_t* seq_lens, int32_t B,
+                        void* o_gated, void* workspace, size_t workspace_bytes,
+                        void* stream);
+
+/* ---------------------------------------------------------------------------
+ * gmla_prefill — causal attention of whole prompts in the explicit form
+ * ("Gated MLA 计算公式" §一, §二): K^(h) = C W_k^(h)T and V^(h) = C W_v^(h)T are
+ * rebuilt from the cached latents, then softmax_{s<=t}(q_t . k_s * scale) V,
+ * gated on the way out.
+ *   q            [T, H, d_h + d_R], packed by sequence
+ *   gate_logits  [T, G] fp32, or NULL for ungated output
+ *   cu_seqlens   [B+1] int32 device prefix sums of the prompt lengths
+ *                (sequence b occupies packed rows cu_seqlens[b] .. cu_seqlens[b+1]-1
+ *                and cache positions 0 .. len-1 of cache slot b)
+ *   T, max_seqlen host copies of cu_seqlens[B] and the longest prompt
+ *   o_gated      [T, H*d_h]
+ *   workspace    device scratch of gmla_prefill_workspace_size(cfg, T, B) bytes
+ * ------------------------------------------------------------------------- */
+GMLA_API gmla_status gmla_prefill(const gmla_config* cfg, const gmla_weights* w,
+                         const void* q, const float* gate_logits,
+                         const gmla_cache* cache, const int32_t* cu_seqlens,
+                         int32_t B, int32_t T, int32_t max_seqlen,
+                         void* o_gated, void* workspace, size_t workspace_bytes,
+                         void* stream);
+
+/* ---------------------------------------------------------------------------
+ * gmla_gate_out — y = W_o [ sigmoid(gate_logits) ⊙ o ] ("Gated MLA 计算公式" §二).
+ *   o            [T, H*d_h]; already gated when gate_logits is NULL
+ *   gate_logits  [T, G] fp32 or NULL
+ *   y            [T, d_model]
+ *   workspace    device scratch of gmla_gate_out_workspace_size(cfg, T) bytes
+ * ------------------------------------------------------------------------- */
+GMLA_API gmla_status gmla_gate_out(const gmla_config* cfg, const gmla_weights* w,
+                          const void* o, int32_t T, const float* gate_logits,
+                          void* y, void* workspace, size_t workspace_bytes,
+                          void* stream);
+
+/* Scratch sizes in bytes (0 is never returned; 256-byte aligned). */
+GMLA_API size_t gmla_latent_project_workspace_size(const gmla_config* cfg, int32_t T);
+GMLA_API size_t gmla_decode_workspace_size(const gmla_config* cfg, int32_t B);
+GMLA_API size_t gmla_prefill_workspace_size(const gmla_config* cfg, int32_t T, int32_t B);
+GMLA_API size_t gmla_gate_out_workspace_size(const gmla_config* cfg, int32_t T);
+
+/* Zero the status word of a workspace (stream-ordered). */
+GMLA_API gmla_status gmla_clear_status(void* workspace, void* stream);
+
+/* Synchronise `stream`, then return the device status word kept in
+ * `workspace` (GMLA_OK, GMLA_ERR_TIMEOUT or GMLA_ERR_DEVICE_RANGE). */
+GMLA_API gmla_status gmla_sync_status(const void* workspace, void* stream);
+
+/* Static description of a status code. */
+GMLA_API const char* gmla_status_string(gmla_status s);
+
+/* Message of the last failing call on this host thread ("" if none). */
+GMLA_API const char* gmla_last_error(void);
+
+/* Library version, e.g. "gmla 0.1.0 sm_100a". */
+GMLA_API const char* gmla_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GMLA_H_ */
