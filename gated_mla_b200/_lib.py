@@ -90,6 +90,10 @@ def _load() -> ctypes.CDLL:
         "gmla_status_string": (ctypes.c_char_p, [st]),
         "gmla_last_error": (ctypes.c_char_p, []),
         "gmla_version": (ctypes.c_char_p, []),
+        "gmla_launch_count": (ctypes.c_uint64, []),
+        "gmla_profile_enable": (st, [I]),
+        "gmla_profile_count": (I, []),
+        "gmla_profile_get": (st, [I, ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(ctypes.c_float)]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -149,3 +153,27 @@ def gmla_clear_status(ws, stream):
 
 def gmla_sync_status(ws, stream):
     return lib.gmla_sync_status(ws, stream)
+
+
+def gmla_launch_count():
+    return lib.gmla_launch_count()
+
+
+def gmla_profile_enable(enable):
+    return lib.gmla_profile_enable(1 if enable else 0)
+
+
+def gmla_profile_count():
+    return lib.gmla_profile_count()
+
+
+def gmla_profile_get(i):
+    """Returns (name, ms) of record i."""
+    name = ctypes.c_char_p()
+    ms = ctypes.c_float()
+    check(lib.gmla_profile_get(i, ctypes.byref(name), ctypes.byref(ms)), "gmla_profile_get")
+    return name.value.decode(), ms.value
+
+
+def profile_records():
+    return [gmla_profile_get(i) for i in range(gmla_profile_count())]

@@ -1,6 +1,6 @@
 """Build libgmla.so (the C-ABI library) in-tree for sm_100a.
 
-    python -m gated_mla_b200.build [--force] [-j N]
+    python gated_mla_b200/build.py [--force] [-j N]
 
 Each .cu under csrc/ compiles to an object with nvcc (arch compute_100a /
 sm_100a, -lineinfo), then one nvcc link makes ``gated_mla_b200/libgmla.so``.

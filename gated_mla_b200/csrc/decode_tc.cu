@@ -673,15 +673,21 @@ static cudaError_t launch_attn(const DecodeArgs& a, cudaStream_t st) {
   auto k = decode_attn_kernel<HG, NBOX>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
+  prof_begin(st, "decode_attn");
   k<<<dim3(a.G, a.n_hg), 192, C::kSmem, st>>>(a);
+  prof_end(st);
   return cudaGetLastError();
 }
 
 cudaError_t launch_decode_bf16(DecodeArgs& a, cudaStream_t st) {
+  prof_begin(st, "decode_plan");
   decode_plan_kernel<<<1, 1024, 0, st>>>(a);
+  prof_end(st);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  prof_begin(st, "decode_absorb");
   decode_absorb_kernel<<<dim3(a.H, (a.B + kAbsorbB - 1) / kAbsorbB), 128, kAbsorbB * a.d_h * sizeof(float), st>>>(a);
+  prof_end(st);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const int nbox = (a.d_c + a.d_rope) / 64;
   switch (a.HG * 16 + nbox) {
@@ -694,7 +700,9 @@ cudaError_t launch_decode_bf16(DecodeArgs& a, cudaStream_t st) {
     default: return cudaErrorInvalidValue;
   }
   if (e != cudaSuccess) return e;
+  prof_begin(st, "decode_merge");
   decode_merge_kernel<<<dim3(a.H, (a.B + kMergeB - 1) / kMergeB), 256, 0, st>>>(a);
+  prof_end(st);
   return cudaGetLastError();
 }
 

@@ -271,7 +271,9 @@ static cudaError_t launch_one(const GemmArgs& a, dim3 grid, cudaStream_t st) {
   auto k = gemm_bf16_tc_kernel<BN, kSwap>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
+  prof_begin(st, kSwap ? "gemm_bf16_swap" : "gemm_bf16");
   k<<<grid, 192, C::kSmemBytes, st>>>(a);
+  prof_end(st);
   return cudaGetLastError();
 }
 

@@ -9,8 +9,10 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 #include <string>
+#include <vector>
 
 #include "../../include/gmla.h"
 #include "common.cuh"
@@ -158,9 +160,44 @@ EpiSeg plain_seg(void* out, int64_t row_stride, int block, int block_stride, int
   return e;
 }
 
+// per-launch timing records
+struct ProfRec {
+  const char* name;
+  cudaEvent_t start, stop;
+};
+std::mutex g_prof_mu;
+bool g_prof_on = false;
+std::vector<ProfRec> g_prof;
+size_t g_prof_used = 0;
+bool g_prof_open = false;
+std::atomic<uint64_t> g_launches{0};
+
 }  // namespace
 
 namespace gmla {
+
+void prof_begin(cudaStream_t st, const char* name) {
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  if (!g_prof_on) return;
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  if (g_prof_used == g_prof.size()) {
+    ProfRec r{};
+    if (cudaEventCreate(&r.start) != cudaSuccess || cudaEventCreate(&r.stop) != cudaSuccess) return;
+    g_prof.push_back(r);
+  }
+  g_prof[g_prof_used].name = name;
+  cudaEventRecord(g_prof[g_prof_used].start, st);
+  g_prof_open = true;
+}
+
+void prof_end(cudaStream_t st) {
+  if (!g_prof_on) return;
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  if (!g_prof_open) return;
+  cudaEventRecord(g_prof[g_prof_used].stop, st);
+  ++g_prof_used;
+  g_prof_open = false;
+}
 
 bool make_tmap_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t row_stride_bytes,
                   uint32_t box_inner, uint32_t box_rows, bool swizzle128) {
@@ -201,6 +238,33 @@ extern "C" {
 const char* gmla_status_string(gmla_status s) { return status_str(s); }
 const char* gmla_last_error(void) { return g_err.c_str(); }
 const char* gmla_version(void) { return "gmla 0.1.0 sm_100a"; }
+
+uint64_t gmla_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+gmla_status gmla_profile_enable(int32_t enable) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  g_prof_on = enable != 0;
+  g_prof_used = 0;
+  g_prof_open = false;
+  return GMLA_OK;
+}
+
+int32_t gmla_profile_count(void) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  return static_cast<int32_t>(g_prof_used);
+}
+
+gmla_status gmla_profile_get(int32_t i, const char** name, float* ms) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  if (i < 0 || static_cast<size_t>(i) >= g_prof_used || !name || !ms)
+    return fail(GMLA_ERR_INVALID_ARG, "profile record %d out of range", i);
+  cudaError_t e = cudaEventSynchronize(g_prof[i].stop);
+  if (e != cudaSuccess) return cuda_fail(e, "gmla_profile_get");
+  e = cudaEventElapsedTime(ms, g_prof[i].start, g_prof[i].stop);
+  if (e != cudaSuccess) return cuda_fail(e, "gmla_profile_get");
+  *name = g_prof[i].name;
+  return GMLA_OK;
+}
 
 size_t gmla_latent_project_workspace_size(const gmla_config* cfg, int32_t T) {
   (void)cfg;

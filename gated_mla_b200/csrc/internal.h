@@ -95,6 +95,12 @@ cudaError_t launch_prefill_attn_bf16(const PrefillArgs& a, cudaStream_t st);
 cudaError_t launch_gate_apply(const void* o, const float* g, void* out, int T, int H, int d_h, int gate_mode,
                               int is_f32, cudaStream_t st);
 
+// ----- instrumentation (gmla.cu) -----
+// Record a start event (when profiling is on) and count one launch.
+void prof_begin(cudaStream_t st, const char* name);
+// Record the matching stop event.
+void prof_end(cudaStream_t st);
+
 // ----- tensor maps -----
 bool make_tmap_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t row_stride_bytes,
                   uint32_t box_inner, uint32_t box_rows, bool swizzle128);

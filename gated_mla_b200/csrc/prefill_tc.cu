@@ -265,7 +265,9 @@ cudaError_t launch_prefill_attn_bf16(const PrefillArgs& a, cudaStream_t st) {
   if (a.d_h != kD) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(prefill_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   if (e != cudaSuccess) return e;
+  prof_begin(st, "prefill_attn");
   prefill_attn_kernel<<<dim3(a.q_tiles_per_seq, a.H, a.B), 192, kSmem, st>>>(a);
+  prof_end(st);
   return cudaGetLastError();
 }
 

@@ -83,7 +83,9 @@ cudaError_t launch_gemm_f32(F32Args a, cudaStream_t st) {
   for (int i = 0; i < a.n_seg; ++i) a.seg_tile_begin[i + 1] = a.seg_tile_begin[i] + (a.seg_rows[i] + kF32FT - 1) / kF32FT;
   const int nx = a.seg_tile_begin[a.n_seg];
   if (nx == 0 || a.T == 0) return cudaSuccess;
+  prof_begin(st, "gemm_f32");
   gemm_f32_kernel<<<dim3(nx, (a.T + kF32TT - 1) / kF32TT), 512, 0, st>>>(a);
+  prof_end(st);
   return cudaGetLastError();
 }
 
@@ -216,7 +218,9 @@ __global__ void __launch_bounds__(kAttnThreads) attn_f32_kernel(const AttnF32Arg
 cudaError_t launch_attn_f32(const AttnF32Args& a, cudaStream_t st) {
   if (a.d_c > kMaxDc || a.d_h + a.d_rope > 512) return cudaErrorInvalidValue;
   if (a.T == 0) return cudaSuccess;
+  prof_begin(st, "attn_f32");
   attn_f32_kernel<<<dim3(a.T, a.H), kAttnThreads, 0, st>>>(a);
+  prof_end(st);
   return cudaGetLastError();
 }
 
@@ -247,8 +251,10 @@ cudaError_t launch_gate_apply(const void* o, const float* g, void* out, int T, i
   if (n == 0) return cudaSuccess;
   const int threads = 256;
   const int64_t blocks = (n + threads - 1) / threads;
+  prof_begin(st, "gate_apply");
   gate_apply_kernel<<<static_cast<int>(blocks < 4096 ? blocks : 4096), threads, 0, st>>>(o, g, out, n, H * d_h, H,
                                                                                            d_h, gate_mode, is_f32);
+  prof_end(st);
   return cudaGetLastError();
 }
 

@@ -211,6 +211,21 @@ GMLA_API const char* gmla_status_string(gmla_status s);
 /* Message of the last failing call on this host thread ("" if none). */
 GMLA_API const char* gmla_last_error(void);
 
+/* ---------------------------------------------------------------------------
+ * Launch accounting and opt-in per-kernel timing (instrumentation, not part of
+ * the method). With profiling enabled, the library records a CUDA event pair
+ * on the launching stream around each of its kernel launches; records are
+ * kept until the next gmla_profile_enable call.
+ * ------------------------------------------------------------------------- */
+/* Kernels launched by this process so far (all devices, all streams). */
+GMLA_API uint64_t gmla_launch_count(void);
+/* Enable (1) or disable (0) per-launch timing; both clear the records. */
+GMLA_API gmla_status gmla_profile_enable(int32_t enable);
+/* Number of recorded launches. */
+GMLA_API int32_t gmla_profile_count(void);
+/* Name and duration (ms) of record i; waits for its stop event. */
+GMLA_API gmla_status gmla_profile_get(int32_t i, const char** name, float* ms);
+
 /* Library version, e.g. "gmla 0.1.0 sm_100a". */
 GMLA_API const char* gmla_version(void);
 

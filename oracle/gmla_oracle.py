@@ -47,7 +47,7 @@ from typing import Optional, Sequence
 import numpy as np
 
 __all__ = [
-    "params", "sigmoid", "rope", "latent", "project", "head_kv",
+    "params", "sigmoid", "rope", "latent", "project", "project_latent", "project_query", "head_kv",
     "attention_explicit", "attention_absorbed", "gate", "output",
     "prefill", "decode", "kv_elements_per_token", "kv_bytes_per_token",
 ]
@@ -120,11 +120,24 @@ def latent(W_c: np.ndarray, x: np.ndarray) -> np.ndarray:
     return x @ W_c.T
 
 
-def project(p: dict, x: np.ndarray, positions: np.ndarray) -> dict:
-    """Everything computed from the tokens' own hidden states x [T, d_model].
+def project_latent(p: dict, x: np.ndarray, positions: np.ndarray) -> dict:
+    """What a token writes into the cache ([MLA-gate] §一; [MLA-notes] §5.2):
 
-    * c  [T, d_c]        latent to cache ([MLA-gate] §一)
-    * kR [T, d_R]        RoPE(W_kr x) at the token's position, cached ([MLA-notes] §5.2)
+    * c  [T, d_c]   latent c = W_c x
+    * kR [T, d_R]   RoPE(W_kr x) at the token's position (shared by all heads)
+    """
+    x = np.asarray(x, dtype=np.float64)
+    out = {"c": latent(p["W_c"], x)}
+    if p["d_R"]:
+        out["kR"] = rope(x @ p["W_kr"].T, positions, p["rope_base"])
+    else:
+        out["kR"] = np.zeros((x.shape[0], 0))
+    return out
+
+
+def project_query(p: dict, x: np.ndarray, positions: np.ndarray) -> dict:
+    """What a token needs as a query:
+
     * q  [T, H, d_h]     q^(h) = W_q^(h) x (reading: full-rank query)
     * qR [T, H, d_R]     RoPE(W_qr^(h) x) at the token's position ([MLA-notes] §5.2)
     * glogit [T, G]      W_g x (+ b_g): gate logits ([MLA-gate] §二 boxed
@@ -134,19 +147,24 @@ def project(p: dict, x: np.ndarray, positions: np.ndarray) -> dict:
     x = np.asarray(x, dtype=np.float64)
     T = x.shape[0]
     H, dh, dR = p["H"], p["d_h"], p["d_R"]
-    out = {"c": latent(p["W_c"], x)}
-    out["q"] = (x @ p["W_q"].T).reshape(T, H, dh)
+    out = {"q": (x @ p["W_q"].T).reshape(T, H, dh)}
     if dR:
-        out["kR"] = rope(x @ p["W_kr"].T, positions, p["rope_base"])
         qr = (x @ p["W_qr"].T).reshape(T, H, dR)
         out["qR"] = rope(qr, np.asarray(positions)[:, None], p["rope_base"])
     else:
-        out["kR"] = np.zeros((T, 0))
         out["qR"] = np.zeros((T, H, 0))
     g = x @ p["W_g"].T
     if p["b_g"] is not None:
         g = g + p["b_g"]
     out["glogit"] = g
+    return out
+
+
+def project(p: dict, x: np.ndarray, positions: np.ndarray) -> dict:
+    """Everything computed from the tokens' own hidden states x [T, d_model]:
+    the cached row (project_latent) and the query side (project_query)."""
+    out = project_latent(p, x, positions)
+    out.update(project_query(p, x, positions))
     return out
 
 
@@ -241,37 +259,43 @@ def prefill(p: dict, x: np.ndarray, lengths: Sequence[int],
 
     x [T, d_model] holds the sequences back to back; ``lengths`` their token
     counts. ``rows`` optionally maps a sequence index to the list of query
-    positions to evaluate (default: all). Returns the intermediates
-    c, kR, q, qR, glogit for all tokens and, for the evaluated rows,
-    ``index`` (packed row ids), o [n, H, d_h], o_tilde, gated and y.
+    positions to evaluate (default: all; sequences not in ``rows`` are
+    evaluated in full). Returns c, kR for all tokens and, for the evaluated
+    rows, ``index`` (packed row ids), q, qR, glogit, o [n, H, d_h], o_tilde,
+    gated and y.
     """
     x = np.asarray(x, dtype=np.float64)
     lengths = [int(L) for L in lengths]
     starts = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int64)
     positions = np.concatenate([np.arange(L) for L in lengths]) if lengths else np.zeros(0, np.int64)
-    pr = project(p, x, positions)
+    lat = project_latent(p, x, positions)
     attn = attention_absorbed if absorbed else attention_explicit
-    idx, o_rows = [], []
     H = p["H"]
+    sel = []
     for b, L in enumerate(lengths):
-        if L == 0:
-            continue
-        t_sel = np.arange(L) if rows is None or b not in rows else np.asarray(sorted(rows[b]))
-        if len(t_sel) == 0:
+        t_sel = np.arange(L) if rows is None or b not in rows else np.asarray(sorted(rows[b]), dtype=np.int64)
+        sel.append(t_sel)
+    index = np.concatenate([starts[b] + t for b, t in enumerate(sel)]) if sel else np.zeros(0, np.int64)
+    qs = project_query(p, x[index], positions[index])
+    o_rows, k = [], 0
+    for b, L in enumerate(lengths):
+        t_sel = sel[b]
+        n = len(t_sel)
+        if n == 0:
             continue
         sl = slice(starts[b], starts[b] + L)
-        C, KR = pr["c"][sl], pr["kR"][sl]
-        gi = starts[b] + t_sel
-        o = np.stack([attn(p, h, pr["q"][gi, h], pr["qR"][gi, h], C, KR, t_sel)
+        C, KR = lat["c"][sl], lat["kR"][sl]
+        o = np.stack([attn(p, h, qs["q"][k:k + n, h], qs["qR"][k:k + n, h], C, KR, t_sel)
                       for h in range(H)], axis=1)              # [n, H, d_h]
-        idx.append(gi)
         o_rows.append(o)
-    out = dict(pr)
-    out["index"] = np.concatenate(idx) if idx else np.zeros(0, np.int64)
+        k += n
+    out = dict(lat)
+    out.update(qs)
+    out["index"] = index
     o = np.concatenate(o_rows) if o_rows else np.zeros((0, H, p["d_h"]))
     out["o"] = o
     out["o_tilde"] = o.reshape(o.shape[0], -1)                 # Concat_h ([MLA-gate] §二)
-    out["gated"] = gate(p, pr["glogit"][out["index"]], out["o_tilde"])
+    out["gated"] = gate(p, qs["glogit"], out["o_tilde"])
     out["y"] = output(p, out["gated"])
     return out
 
