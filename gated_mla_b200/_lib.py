@@ -79,6 +79,7 @@ def _load() -> ctypes.CDLL:
     sig = {
         "gmla_latent_project": (st, [cfgp, wp, P, I, P, P, cp, P, P, P, S, P]),
         "gmla_decode": (st, [cfgp, wp, P, P, cp, P, I, P, P, S, P]),
+        "gmla_decode_noalloc": (st, [cfgp, wp, P, P, cp, P, I, P, P]),
         "gmla_prefill": (st, [cfgp, wp, P, P, cp, P, I, I, I, P, P, S, P]),
         "gmla_gate_out": (st, [cfgp, wp, P, I, P, P, P, S, P]),
         "gmla_latent_project_workspace_size": (S, [cfgp, I]),
@@ -120,6 +121,11 @@ def gmla_latent_project(cfg, w, x, T, positions, seq_ids, cache, q_out, gate_log
 def gmla_decode(cfg, w, q, gate_logits, cache, seq_lens, B, o, ws, ws_bytes, stream):
     return lib.gmla_decode(ctypes.byref(cfg), ctypes.byref(w), q, gate_logits, ctypes.byref(cache),
                            seq_lens, B, o, ws, ws_bytes, stream)
+
+
+def gmla_decode_noalloc(cfg, w, q, gate_logits, cache, seq_lens, B, o, stream):
+    return lib.gmla_decode_noalloc(ctypes.byref(cfg), ctypes.byref(w), q, gate_logits, ctypes.byref(cache),
+                                   seq_lens, B, o, stream)
 
 
 def gmla_prefill(cfg, w, q, gate_logits, cache, cu_seqlens, B, T, max_seqlen, o, ws, ws_bytes, stream):

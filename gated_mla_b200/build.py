@@ -22,7 +22,7 @@ CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 BUILD = os.path.join(ROOT, "_build", "gmla")
 LIB = os.path.join(HERE, "libgmla.so")
-SOURCES = ["gmla.cu", "gemm_tc.cu", "decode_tc.cu", "prefill_tc.cu", "simt_f32.cu"]
+SOURCES = ["gmla.cu", "gemm_tc.cu", "decode_tc.cu", "prefill_tc.cu", "simt_f32.cu", "noalloc.cu"]
 HEADERS = ["ptx.cuh", "common.cuh", "internal.h"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -176,6 +176,8 @@ std::atomic<uint64_t> g_launches{0};
 
 namespace gmla {
 
+void set_last_error(const char* msg) { g_err = msg ? msg : ""; }
+
 void prof_begin(cudaStream_t st, const char* name) {
   g_launches.fetch_add(1, std::memory_order_relaxed);
   if (!g_prof_on) return;

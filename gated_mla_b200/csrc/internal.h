@@ -95,6 +95,9 @@ cudaError_t launch_prefill_attn_bf16(const PrefillArgs& a, cudaStream_t st);
 cudaError_t launch_gate_apply(const void* o, const float* g, void* out, int T, int H, int d_h, int gate_mode,
                               int is_f32, cudaStream_t st);
 
+// ----- error message of the current host thread (gmla.cu) -----
+void set_last_error(const char* msg);
+
 // ----- instrumentation (gmla.cu) -----
 // Record a start event (when profiling is on) and count one launch.
 void prof_begin(cudaStream_t st, const char* name);

@@ -192,6 +192,29 @@ GMLA_API gmla_status gmla_gate_out(const gmla_config* cfg, const gmla_weights* w
                           void* y, void* workspace, size_t workspace_bytes,
                           void* stream);
 
+/* ---------------------------------------------------------------------------
+ * gmla_decode_noalloc — gmla_decode for callers that cannot allocate device
+ * memory: code running under CUDA graph capture (cudaMalloc is not allowed
+ * there), engines and plugins whose device memory belongs to their own pool,
+ * and loops that cannot pay cudaMalloc's implicit synchronisation. The pages
+ * have no counterpart to this call: it is a deployment convenience.
+ * Same arguments and results as gmla_decode, minus the workspace: the scratch
+ * is a 16 MiB array in the library's device memory, held by every GPU that
+ * loads the library until the process exits. The call allocates nothing.
+ *   - Batches whose gmla_decode_workspace_size() exceeds 16 MiB are rejected
+ *     with GMLA_ERR_WORKSPACE (use gmla_decode with a workspace instead).
+ *   - The first call on a device looks up the array's device address; make
+ *     that first call before any stream capture.
+ *   - All calls share the array and it keeps the previous call's contents:
+ *     calls whose kernels overlap on the GPU race on it, so serialise them.
+ *   - Device-side faults are recorded in the shared array's status word,
+ *     which each call clears first; this variant does not report them back.
+ * ------------------------------------------------------------------------- */
+GMLA_API gmla_status gmla_decode_noalloc(const gmla_config* cfg, const gmla_weights* w,
+                                         const void* q, const float* gate_logits,
+                                         const gmla_cache* cache, const int32_t* seq_lens,
+                                         int32_t B, void* o_gated, void* stream);
+
 /* Scratch sizes in bytes (0 is never returned; 256-byte aligned). */
 GMLA_API size_t gmla_latent_project_workspace_size(const gmla_config* cfg, int32_t T);
 GMLA_API size_t gmla_decode_workspace_size(const gmla_config* cfg, int32_t B);
