@@ -21,7 +21,7 @@ struct CacheView {
 };
 
 // Global row index of token `pos` of sequence `b`, or -1 when out of range.
-__device__ __forceinline__ int64_t cache_row(const CacheView& c, int b, int pos) {
+static __device__ __noinline__ int64_t cache_row(const CacheView& c, int b, int pos) {
   if (b < 0 || pos < 0) return -1;
   if (!c.paged) {
     if (b >= c.batch || pos >= c.capacity) return -1;
@@ -50,6 +50,10 @@ struct EpiSeg {
   int32_t out_f32;       // 1: fp32 output, 0: bf16 output
   int32_t rope;
   int32_t cache_scatter;
+  // optional sigmoid gate: v *= sigmoid(gate[t * gate_stride + f / gate_div])
+  const float* gate;
+  int32_t gate_stride;
+  int32_t gate_div;
 };
 
 constexpr int kMaxSeg = 5;
@@ -63,11 +67,22 @@ struct GemmArgs {
   int32_t n_seg;
   int32_t T;
   int32_t K;
+  // row_mode 2: per-group activations (swap orientation): the weight rows of
+  //   group g = wrow / rows_per_group read activation rows g*act_group_stride + token.
+  int32_t rows_per_group;
+  int32_t act_group_stride;
   // row_mode 0: token tile y covers packed tokens [y*tile, ...).
   // row_mode 1: prefill sequence tiles: y -> (sequence y / tiles_per_seq,
   //   offset (y % tiles_per_seq) * tile); activation rows start at
   //   sequence * act_seq_stride, packed tokens at cu_seqlens[sequence].
   int32_t row_mode;
+  // split-K (swap orientation only): blockIdx.z is the split; each split
+  // accumulates kb_per_split 64-wide K blocks, writes an fp32 partial tile and
+  // the last split to finish (ticket in counters[tile]) sums and stores.
+  int32_t splits;
+  int32_t kb_per_split;
+  float* partial;            // [splits][tiles][BN][128] fp32
+  int32_t* counters;         // [tiles], zero before the launch
   int32_t tiles_per_seq;
   int32_t act_seq_stride;
   const int32_t* cu_seqlens;
@@ -81,8 +96,8 @@ struct GemmArgs {
 // RoPE of one element given its pair partner: pair (x0, x1) at feature
 // (2i, 2i+1) becomes (x0 cos - x1 sin, x0 sin + x1 cos), angle pos * base^(-2i/d).
 // The angle is formed and reduced in double so long positions keep their accuracy.
-__device__ __forceinline__ float rope_rotate(float v, float partner, bool odd, int pos, int i_pair, int d,
-                                             double log2_base) {
+static __device__ __noinline__ float rope_rotate(float v, float partner, bool odd, int pos, int i_pair, int d,
+                                          double log2_base) {
   const double inv = exp2(-(2.0 * i_pair / d) * log2_base);
   double ang = static_cast<double>(pos) * inv;
   ang -= 6.283185307179586476925 * rint(ang * 0.159154943091895335768883763);
@@ -91,7 +106,8 @@ __device__ __forceinline__ float rope_rotate(float v, float partner, bool odd, i
   return odd ? (partner * s + v * c) : (v * c - partner * s);
 }
 
-__device__ __forceinline__ void epi_store(const EpiSeg& e, int64_t row, int f, float v) {
+__device__ __forceinline__ void epi_store(const EpiSeg& e, int64_t row, int f, float v, int t = 0) {
+  if (e.gate) v *= 1.f / (1.f + __expf(-e.gate[static_cast<int64_t>(t) * e.gate_stride + f / e.gate_div]));
   const int64_t off = row * e.row_stride + static_cast<int64_t>(f / e.block) * e.block_stride + (f % e.block) +
                       e.col_offset;
   if (e.bias) v += e.bias[f];

@@ -34,8 +34,8 @@ constexpr int kNcBox = kDc / 64;
 // ---------------------------------------------------------------------------
 // 1. plan
 // ---------------------------------------------------------------------------
-// Exclusive prefix sum over a block of 1024 threads; *total gets the sum.
-__device__ __forceinline__ int block_excl_scan_1024(int v, int* s_warp, int* total) {
+// Exclusive prefix sum over the block (blockDim a multiple of 32); *total gets the sum.
+__device__ __forceinline__ int block_excl_scan(int v, int* s_warp, int* total) {
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   int inc = v;
 #pragma unroll
@@ -46,7 +46,7 @@ __device__ __forceinline__ int block_excl_scan_1024(int v, int* s_warp, int* tot
   if (lane == 31) s_warp[w] = inc;
   __syncthreads();
   if (w == 0) {
-    const int x = s_warp[lane];
+    const int x = lane < static_cast<int>(blockDim.x >> 5) ? s_warp[lane] : 0;
     int y = x;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -65,7 +65,7 @@ __device__ __forceinline__ int block_excl_scan_1024(int v, int* s_warp, int* tot
 // Tiles of 128 tokens of all sequences, concatenated, are cut into G equal
 // ranges (one per CTA of a head group). A segment is the part of one sequence
 // inside one range; seg_info = {sequence, first tile, end tile, CTA}.
-__global__ void __launch_bounds__(1024) decode_plan_kernel(DecodeArgs a) {
+__device__ void decode_plan_block(const DecodeArgs& a) {
   __shared__ int s_warp[32];
   __shared__ int s_total;
   __shared__ int s_sum;
@@ -91,14 +91,14 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(DecodeArgs a) {
     if (L < 0 || L > limit || b >= a.cache.batch) L = 0;
     const int t = (L + kTileTok - 1) / kTileTok;
     int tsum, ssum;
-    const int P = tile_carry + block_excl_scan_1024(t, s_warp, &s_total);
+    const int P = tile_carry + block_excl_scan(t, s_warp, &s_total);
     tsum = s_total;
     int nseg = 0, g_first = 0;
     if (t > 0) {
       g_first = P / tpc;
       nseg = (P + t - 1) / tpc - g_first + 1;
     }
-    const int S = seg_carry + block_excl_scan_1024(nseg, s_warp, &s_total);
+    const int S = seg_carry + block_excl_scan(nseg, s_warp, &s_total);
     ssum = s_total;
     if (b < a.B) {
       a.seq_first_seg[b] = S;
@@ -119,59 +119,87 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(DecodeArgs a) {
 
 // ---------------------------------------------------------------------------
 // 2. absorb: qa[b, h, :d_c] = bf16(q_scale * W_k^(h)T q^(h)), qa[b, h, d_c:] = bf16(q_scale * q^R)
+//    One block per (head, 8 sequences, 64 latent columns); the d_h sum is split
+//    over 16 thread groups and reduced in shared memory. The last block of the
+//    grid runs the split plan instead.
 // ---------------------------------------------------------------------------
 constexpr int kAbsorbB = 8;
+constexpr int kAbsorbCols = 64;
+constexpr int kAbsorbKG = 16;
 
-__global__ void __launch_bounds__(128) decode_absorb_kernel(DecodeArgs a) {
-  const int h = blockIdx.x;
-  const int b0 = blockIdx.y * kAbsorbB;
+__global__ void __launch_bounds__(256) decode_absorb_plan_kernel(DecodeArgs a) {
+  const int n_cblk = a.d_c / kAbsorbCols;
+  const int n_bblk = (a.B + kAbsorbB - 1) / kAbsorbB;
+  const int blk = blockIdx.x;
+  if (blk == a.H * n_bblk * n_cblk) {
+    decode_plan_block(a);
+    return;
+  }
+  const int h = blk / (n_bblk * n_cblk);
+  const int rem = blk % (n_bblk * n_cblk);
+  const int b0 = (rem / n_cblk) * kAbsorbB;
+  const int cb = rem % n_cblk;
   const int nb = min(kAbsorbB, a.B - b0);
   const int dq = a.d_h + a.d_rope;
   const int row = a.d_c + a.d_rope;
-  extern __shared__ float sq[];   // [kAbsorbB][d_h]
+  __shared__ float sq[kAbsorbB][256];
+  __shared__ float red[kAbsorbKG][kAbsorbB][kAbsorbCols];
   const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(a.q);
   for (int i = threadIdx.x; i < kAbsorbB * a.d_h; i += blockDim.x) {
     const int bi = i / a.d_h, k = i % a.d_h;
-    sq[i] = bi < nb ? __bfloat162float(q[(static_cast<int64_t>(b0 + bi) * a.H + h) * dq + k]) : 0.f;
+    sq[bi][k] = bi < nb ? __bfloat162float(q[(static_cast<int64_t>(b0 + bi) * a.H + h) * dq + k]) : 0.f;
   }
   __syncthreads();
+  const int kg = threadIdx.x >> 4;             // 16 groups over d_h
+  const int cl = (threadIdx.x & 15) * 4;       // 4 columns of the block's 64
+  const int c0 = cb * kAbsorbCols + cl;
+  const int kper = (a.d_h + kAbsorbKG - 1) / kAbsorbKG;
   const __nv_bfloat16* Wk = static_cast<const __nv_bfloat16*>(a.W_k) + static_cast<int64_t>(h) * a.d_h * a.d_c;
-  __nv_bfloat16* qa = static_cast<__nv_bfloat16*>(a.qa);
-  // each thread: 4 consecutive latent columns
-  for (int c0 = threadIdx.x * 4; c0 < a.d_c; c0 += blockDim.x * 4) {
-    float acc[kAbsorbB][4];
+  float acc[kAbsorbB][4];
 #pragma unroll
-    for (int bi = 0; bi < kAbsorbB; ++bi)
+  for (int bi = 0; bi < kAbsorbB; ++bi)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) acc[bi][j] = 0.f;
-    for (int k = 0; k < a.d_h; ++k) {
-      const uint2 wv = *reinterpret_cast<const uint2*>(Wk + static_cast<int64_t>(k) * a.d_c + c0);
-      const __nv_bfloat162 w01 = *reinterpret_cast<const __nv_bfloat162*>(&wv.x);
-      const __nv_bfloat162 w23 = *reinterpret_cast<const __nv_bfloat162*>(&wv.y);
-      const float w[4] = {__low2float(w01), __high2float(w01), __low2float(w23), __high2float(w23)};
+    for (int j = 0; j < 4; ++j) acc[bi][j] = 0.f;
+  const int k_lo = kg * kper, k_hi = min(a.d_h, k_lo + kper);
+  uint2 wv[16];
 #pragma unroll
-      for (int bi = 0; bi < kAbsorbB; ++bi) {
-        const float qk = sq[bi * a.d_h + k];
+  for (int i = 0; i < 16; ++i)
+    if (k_lo + i < k_hi) wv[i] = *reinterpret_cast<const uint2*>(Wk + static_cast<int64_t>(k_lo + i) * a.d_c + c0);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[bi][j] = fmaf(qk, w[j], acc[bi][j]);
-      }
-    }
+  for (int i = 0; i < 16; ++i) {
+    if (k_lo + i >= k_hi) break;
+    const __nv_bfloat162 w01 = *reinterpret_cast<const __nv_bfloat162*>(&wv[i].x);
+    const __nv_bfloat162 w23 = *reinterpret_cast<const __nv_bfloat162*>(&wv[i].y);
+    const float w[4] = {__low2float(w01), __high2float(w01), __low2float(w23), __high2float(w23)};
 #pragma unroll
     for (int bi = 0; bi < kAbsorbB; ++bi) {
-      if (bi >= nb) break;
-      __nv_bfloat16* dst = qa + (static_cast<int64_t>(b0 + bi) * a.H + h) * row + c0;
-      uint2 pk;
-      pk.x = pack_bf16x2(acc[bi][0] * a.q_scale, acc[bi][1] * a.q_scale);
-      pk.y = pack_bf16x2(acc[bi][2] * a.q_scale, acc[bi][3] * a.q_scale);
-      *reinterpret_cast<uint2*>(dst) = pk;
+      const float qk = sq[bi][k_lo + i];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[bi][j] = fmaf(qk, w[j], acc[bi][j]);
     }
   }
+#pragma unroll
+  for (int bi = 0; bi < kAbsorbB; ++bi)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) red[kg][bi][cl + j] = acc[bi][j];
+  __syncthreads();
+  __nv_bfloat16* qa = static_cast<__nv_bfloat16*>(a.qa);
+  for (int o = threadIdx.x; o < kAbsorbB * kAbsorbCols; o += blockDim.x) {
+    const int bi = o / kAbsorbCols, c = o % kAbsorbCols;
+    if (bi >= nb) continue;
+    float v = 0.f;
+#pragma unroll
+    for (int g = 0; g < kAbsorbKG; ++g) v += red[g][bi][c];
+    qa[(static_cast<int64_t>(b0 + bi) * a.H + h) * row + cb * kAbsorbCols + c] = __float2bfloat16_rn(v * a.q_scale);
+  }
   // decoupled RoPE query dims: copied (already rotated), scaled
-  for (int i = threadIdx.x; i < nb * a.d_rope; i += blockDim.x) {
-    const int bi = i / a.d_rope, r = i % a.d_rope;
-    const int64_t src = (static_cast<int64_t>(b0 + bi) * a.H + h) * dq + a.d_h + r;
-    qa[(static_cast<int64_t>(b0 + bi) * a.H + h) * row + a.d_c + r] =
-        __float2bfloat16_rn(__bfloat162float(q[src]) * a.q_scale);
+  if (cb == 0) {
+    for (int i = threadIdx.x; i < nb * a.d_rope; i += blockDim.x) {
+      const int bi = i / a.d_rope, r = i % a.d_rope;
+      const int64_t src = (static_cast<int64_t>(b0 + bi) * a.H + h) * dq + a.d_h + r;
+      qa[(static_cast<int64_t>(b0 + bi) * a.H + h) * row + a.d_c + r] =
+          __float2bfloat16_rn(__bfloat162float(q[src]) * a.q_scale);
+    }
   }
 }
 
@@ -543,98 +571,36 @@ __global__ void __launch_bounds__(192, 1) decode_attn_kernel(const __grid_consta
 }
 
 // ---------------------------------------------------------------------------
-// 4. merge partials, W_v up-projection, sigmoid gate
+// 4. merge the split-K partials of each (head, sequence) by their log-sum-exp
+//    weights: O_lat = sum_i 2^(m_i - m) O_i / sum_i 2^(m_i - m) l_i, written as
+//    bf16 [H, B, d_c] for the W_v product (a tensor-core GEMM with the gate in
+//    its epilogue). Block (0, 0) also clears that GEMM's split-K tickets.
 // ---------------------------------------------------------------------------
-constexpr int kMergeB = 4;
-
-__global__ void __launch_bounds__(256) decode_merge_kernel(DecodeArgs a) {
-  const int h = blockIdx.x;
-  const int b0 = blockIdx.y * kMergeB;
-  const int nb = min(kMergeB, a.B - b0);
+__global__ void __launch_bounds__(128) decode_merge_kernel(DecodeArgs a) {
+  const int h = blockIdx.x, b = blockIdx.y;
   const int hg = h / a.HG, hl = h % a.HG;
-  __shared__ float olat[kMergeB][kDc];
-  __shared__ float mx_s[kMergeB];
-  __shared__ float inv_l[kMergeB];
-  const int tid = threadIdx.x;
+  if (h == 0 && b == 0)
+    for (int i = threadIdx.x; i < a.n_gemm_tiles; i += blockDim.x) a.gemm_counters[i] = 0;
+  const int s0 = a.seq_first_seg[b], s1 = a.seq_first_seg[b + 1];
   const int64_t base = static_cast<int64_t>(hg) * a.max_seg;
-  // m = max_i m_i, l = sum_i 2^(m_i - m) l_i over the segments of each sequence
-  if (tid < 32 * kMergeB) {
-    const int bi = tid >> 5, ln = tid & 31;
-    if (bi < nb) {
-      const int b = b0 + bi;
-      const int s0 = a.seq_first_seg[b], s1 = a.seq_first_seg[b + 1];
-      float mx = -__int_as_float(0x7f800000);
-      for (int s = s0 + ln; s < s1; s += 32) mx = fmaxf(mx, a.ml_part[((base + s) * a.HG + hl) * 2]);
-      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      float l = 0.f;
-      for (int s = s0 + ln; s < s1; s += 32) {
-        const float* ml = a.ml_part + ((base + s) * a.HG + hl) * 2;
-        l += ex2_approx(ml[0] - mx) * ml[1];
-      }
-      for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-      if (ln == 0) {
-        mx_s[bi] = mx;
-        inv_l[bi] = (s1 > s0 && l > 0.f) ? 1.f / l : 0.f;
-      }
-    }
+  float mx = -__int_as_float(0x7f800000);
+  for (int s = s0; s < s1; ++s) mx = fmaxf(mx, a.ml_part[((base + s) * a.HG + hl) * 2]);
+  float l = 0.f;
+  float acc[kDc / 128];
+#pragma unroll
+  for (int j = 0; j < kDc / 128; ++j) acc[j] = 0.f;
+  for (int s = s0; s < s1; ++s) {
+    const float* ml = a.ml_part + ((base + s) * a.HG + hl) * 2;
+    const float w = ex2_approx(ml[0] - mx);
+    l = fmaf(w, ml[1], l);
+    const float* op = a.o_part + ((base + s) * a.HG + hl) * kDc;
+#pragma unroll
+    for (int j = 0; j < kDc / 128; ++j) acc[j] = fmaf(w, __ldcg(op + j * 128 + threadIdx.x), acc[j]);
   }
-  __syncthreads();
-  // O_lat = sum_i 2^(m_i - m) O_i / l
-  for (int i = tid; i < kMergeB * kDc; i += blockDim.x) {
-    const int bi = i / kDc, d = i % kDc;
-    float acc = 0.f;
-    if (bi < nb) {
-      const int b = b0 + bi;
-      const int s0 = a.seq_first_seg[b], s1 = a.seq_first_seg[b + 1];
-      for (int s = s0; s < s1; ++s) {
-        const float w = ex2_approx(a.ml_part[((base + s) * a.HG + hl) * 2] - mx_s[bi]);
-        acc = fmaf(w, a.o_part[((base + s) * a.HG + hl) * kDc + d], acc);
-      }
-      acc *= inv_l[bi];
-    }
-    olat[bi][d] = acc;
-  }
-  __syncthreads();
-  // o[b, h*d_h + i] = sum_d W_v[h, i, d] * olat[b, d]; one warp per output row i
-  const __nv_bfloat16* Wv = static_cast<const __nv_bfloat16*>(a.W_v) + static_cast<int64_t>(h) * a.d_h * kDc;
-  const int warp = tid >> 5, lane = tid & 31;
-  __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.o);
-  const int HD = a.H * a.d_h;
-  const int G = a.gate_mode == 0 ? HD : a.H;
-  for (int i = warp; i < a.d_h; i += blockDim.x / 32) {
-    float acc[kMergeB];
+  const float inv = (s1 > s0 && l > 0.f) ? 1.f / l : 0.f;
+  __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.olat) + (static_cast<int64_t>(h) * a.B + b) * kDc;
 #pragma unroll
-    for (int bi = 0; bi < kMergeB; ++bi) acc[bi] = 0.f;
-    const __nv_bfloat16* wr = Wv + static_cast<int64_t>(i) * kDc;
-#pragma unroll
-    for (int it = 0; it < kDc / 256; ++it) {
-      const int d0 = it * 256 + lane * 8;
-      const uint4 wv = *reinterpret_cast<const uint4*>(wr + d0);
-      const __nv_bfloat162* w2 = reinterpret_cast<const __nv_bfloat162*>(&wv);
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float wa = __low2float(w2[k]), wb = __high2float(w2[k]);
-#pragma unroll
-        for (int bi = 0; bi < kMergeB; ++bi)
-          acc[bi] = fmaf(wa, olat[bi][d0 + 2 * k], fmaf(wb, olat[bi][d0 + 2 * k + 1], acc[bi]));
-      }
-    }
-#pragma unroll
-    for (int bi = 0; bi < kMergeB; ++bi)
-      for (int o = 16; o > 0; o >>= 1) acc[bi] += __shfl_xor_sync(0xffffffffu, acc[bi], o);
-    if (lane < nb) {
-      const int b = b0 + lane;
-      float v = 0.f;
-#pragma unroll
-      for (int bi = 0; bi < kMergeB; ++bi)
-        if (bi == lane) v = acc[bi];
-      if (a.gate_logits) {
-        const float z = a.gate_logits[static_cast<int64_t>(b) * G + (a.gate_mode == 0 ? h * a.d_h + i : h)];
-        v *= 1.f / (1.f + __expf(-z));
-      }
-      out[static_cast<int64_t>(b) * HD + h * a.d_h + i] = __float2bfloat16_rn(v);
-    }
-  }
+  for (int j = 0; j < kDc / 128; ++j) dst[j * 128 + threadIdx.x] = __float2bfloat16_rn(acc[j] * inv);
 }
 
 // ---------------------------------------------------------------------------
@@ -642,7 +608,7 @@ __global__ void __launch_bounds__(256) decode_merge_kernel(DecodeArgs a) {
 // ---------------------------------------------------------------------------
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-DecodeLayout decode_layout(int B, int H, int d_c, int d_rope, int num_sms) {
+DecodeLayout decode_layout(int B, int H, int d_h, int d_c, int d_rope, int num_sms) {
   DecodeLayout L{};
   L.HG = H <= 16 ? 16 : (H % 64 == 0 ? 64 : (H % 32 == 0 ? 32 : 16));
   L.n_hg = (H + L.HG - 1) / L.HG;
@@ -663,6 +629,11 @@ DecodeLayout decode_layout(int B, int H, int d_c, int d_rope, int num_sms) {
   off = align256(off + static_cast<size_t>(B + 1) * 4);
   L.off_ctafirst = off;
   off = align256(off + static_cast<size_t>(L.G + 1) * 4);
+  L.off_olat = off;
+  off = align256(off + static_cast<size_t>(H) * B * d_c * 2);
+  L.off_gemm = off;
+  L.gemm_plan = gemm_swap_plan(H * d_h / 128, B, d_c, num_sms);
+  off = align256(off + L.gemm_plan.ws_bytes);
   L.total = off;
   return L;
 }
@@ -680,15 +651,12 @@ static cudaError_t launch_attn(const DecodeArgs& a, cudaStream_t st) {
 }
 
 cudaError_t launch_decode_bf16(DecodeArgs& a, cudaStream_t st) {
-  prof_begin(st, "decode_plan");
-  decode_plan_kernel<<<1, 1024, 0, st>>>(a);
+  const int n_absorb = a.H * ((a.B + kAbsorbB - 1) / kAbsorbB) * (a.d_c / kAbsorbCols);
+  prof_begin(st, "decode_absorb_plan");
+  decode_absorb_plan_kernel<<<n_absorb + 1, 256, 0, st>>>(a);
   prof_end(st);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  prof_begin(st, "decode_absorb");
-  decode_absorb_kernel<<<dim3(a.H, (a.B + kAbsorbB - 1) / kAbsorbB), 128, kAbsorbB * a.d_h * sizeof(float), st>>>(a);
-  prof_end(st);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const int nbox = (a.d_c + a.d_rope) / 64;
   switch (a.HG * 16 + nbox) {
     case 16 * 16 + 8: e = launch_attn<16, 8>(a, st); break;
@@ -701,7 +669,7 @@ cudaError_t launch_decode_bf16(DecodeArgs& a, cudaStream_t st) {
   }
   if (e != cudaSuccess) return e;
   prof_begin(st, "decode_merge");
-  decode_merge_kernel<<<dim3(a.H, (a.B + kMergeB - 1) / kMergeB), 256, 0, st>>>(a);
+  decode_merge_kernel<<<dim3(a.H, a.B), 128, 0, st>>>(a);
   prof_end(st);
   return cudaGetLastError();
 }

@@ -26,9 +26,10 @@ struct GemmCfg {
   static constexpr int kABytes = 128 * 128;              // 128 rows x 64 bf16
   static constexpr int kBBytes = BN * 128;               // BN rows x 64 bf16
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kStages = (BN >= 256) ? 4 : (BN >= 128 ? 6 : 8);
+  // narrow tiles (few tokens, weight streaming): 4 stages so two CTAs share an SM
+  static constexpr int kStages = (BN >= 256) ? 4 : (BN >= 128 ? 6 : 4);
   static constexpr int kTmemCols = BN < 32 ? 32 : BN;
-  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/ + 12 * BN;
 };
 
 struct GemmTile {
@@ -51,6 +52,10 @@ __device__ __forceinline__ bool gemm_tile(const GemmArgs& a, GemmTile& t) {
   if (a.row_mode == 0) {
     t.tok0 = blockIdx.y * kTTile;
     t.act_row0 = t.tok0;
+    t.ntok = min(kTTile, a.T - t.tok0);
+  } else if (a.row_mode == 2) {
+    t.tok0 = blockIdx.y * kTTile;
+    t.act_row0 = (a.seg_tile_begin[s] * kWTile + t.wrow0) / a.rows_per_group * a.act_group_stride + t.tok0;
     t.ntok = min(kTTile, a.T - t.tok0);
   } else {
     // prefill sequence tiles: token tile -> (sequence, offset)
@@ -75,12 +80,23 @@ __global__ void __launch_bounds__(192, 1) gemm_bf16_tc_kernel(const __grid_const
   uint64_t* drain = acc_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* last_flag = abort_flag + 1;
+  // per-token output row and position of this tile (swap orientation), filled once
+  int64_t* tok_row = reinterpret_cast<int64_t*>(smem + C::kStages * C::kStageBytes + 256);
+  int* tok_pos = reinterpret_cast<int*>(tok_row + (kSwap ? BN : 1));
 
   GemmTile tile;
   if (!gemm_tile<BN, kSwap>(a, tile)) return;   // uniform across the block
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int num_kb = (a.K + 63) / 64;
+  if (threadIdx.x == 0) {   // start the descriptor fetches while the block sets up
+    tma_prefetch_desc(&a.act);
+    tma_prefetch_desc(&a.wt[tile.seg]);
+  }
+  const int num_kb_total = (a.K + 63) / 64;
+  const int kbps = (kSwap && a.kb_per_split > 0) ? a.kb_per_split : num_kb_total;
+  const int kb_begin = kSwap ? blockIdx.z * kbps : 0;
+  const int num_kb = kSwap ? min(num_kb_total - kb_begin, kbps) : num_kb_total;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::kStages; ++i) {
@@ -118,8 +134,8 @@ __global__ void __launch_bounds__(192, 1) gemm_bf16_tc_kernel(const __grid_const
         uint8_t* sb = sa + C::kABytes;
         mbar_arrive_expect_tx(&full[st], C::kStageBytes);
         if (kSwap) {
-          tma_load_2d(wmap, &full[st], sa, kb * 64, tile.wrow0, pol_w);
-          tma_load_2d(&a.act, &full[st], sb, kb * 64, tile.act_row0, pol_x);
+          tma_load_2d(wmap, &full[st], sa, (kb_begin + kb) * 64, tile.wrow0, pol_w);
+          tma_load_2d(&a.act, &full[st], sb, (kb_begin + kb) * 64, tile.act_row0, pol_x);
         } else {
           tma_load_2d(&a.act, &full[st], sa, kb * 64, tile.act_row0, pol_x);
           tma_load_2d(wmap, &full[st], sb, kb * 64, tile.wrow0, pol_w);
@@ -162,41 +178,131 @@ __global__ void __launch_bounds__(192, 1) gemm_bf16_tc_kernel(const __grid_const
     // epilogue warps 2..5 -> TMEM lane quarter (warp % 4)
     const int q = warp & 3;
     const int r = q * 32 + lane;            // accumulator row of this thread
-    if (mbar_wait(acc_full, 0, abort_flag, a.status)) {
+    // Split-K epilogues meet at named barrier 2; a failed wait still walks the
+    // same barriers (with its stores skipped) so the four warps stay in step.
+    const bool acc_ok = mbar_wait(acc_full, 0, abort_flag, a.status);
+    if (acc_ok || kSwap) {
       tc_fence_after();
-      const EpiSeg& e = a.epi[tile.seg];
+      // by value: a runtime-indexed reference into the parameter space costs a
+      // chain of constant-bank loads on every use
+      const EpiSeg e = a.epi[tile.seg];
       const int seg_rows = a.seg_rows[tile.seg];
       if (kSwap) {
-        // row r = weight feature, columns = tokens
+        // row r = weight feature, columns = tokens. The tile's token -> output
+        // row / position table is built once in shared memory so the store loop
+        // has no dependent global loads.
         const int f = tile.wrow0 + r;
-#pragma unroll 1
-        for (int c0 = 0; c0 < BN; c0 += 16) {
-          uint32_t v[16];
-          tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + c0, v);
-          tmem_ld_wait();
-#pragma unroll
+        for (int lt = threadIdx.x - 64; lt < BN; lt += 128) {
+          const int tok = tile.tok0 + lt;
+          int64_t row = tok;
+          int pos = 0;
+          if (lt < tile.ntok && (e.rope || e.cache_scatter)) pos = a.positions[tok];
+          if (lt < tile.ntok && e.cache_scatter) {
+            row = cache_row(a.cache, a.seq_ids[tok], pos);
+            if (row < 0) report_status(a.status, kStatusRange);
+          }
+          tok_row[lt] = lt < tile.ntok ? row : -1;
+          tok_pos[lt] = pos;
+        }
+        asm volatile("bar.sync 2, 128;" ::: "memory");
+        // this thread's feature is fixed: hoist its column offset, bias and gate index
+        const int64_t colpart =
+            static_cast<int64_t>(f / e.block) * e.block_stride + (f % e.block) + e.col_offset;
+        const bool f_ok = f < seg_rows;
+        const float fbias = (e.bias && f_ok) ? e.bias[f] : 0.f;
+        const int gcol = e.gate ? f / e.gate_div : 0;
+        auto store_chunk = [&](int c0, float (&x)[16]) {
+#pragma unroll 4
           for (int j = 0; j < 16; ++j) {
             const int tl = c0 + j;
-            float val = __uint_as_float(v[j]);
-            const int tok = tile.tok0 + tl;
-            const bool tok_ok = tl < tile.ntok;
-            int pos = 0;
-            if (e.rope || e.cache_scatter) pos = tok_ok ? a.positions[tok] : 0;
+            float val = x[j];
             if (e.rope) {
               const float partner = __shfl_xor_sync(0xffffffffu, val, 1);
               const int fi = f % e.block;
-              val = rope_rotate(val, partner, fi & 1, pos, fi >> 1, e.block, a.log2_rope_base);
+              val = rope_rotate(val, partner, fi & 1, tok_pos[tl], fi >> 1, e.block, a.log2_rope_base);
             }
-            if (!tok_ok || f >= seg_rows) continue;
-            int64_t row = tok;
-            if (e.cache_scatter) {
-              row = cache_row(a.cache, a.seq_ids[tok], pos);
-              if (row < 0) {
-                report_status(a.status, kStatusRange);
-                continue;
+            const int64_t row = tok_row[tl];
+            if (row < 0 || !f_ok) continue;
+            val += fbias;
+            if (e.gate)
+              val *= 1.f / (1.f + __expf(-e.gate[static_cast<int64_t>(tile.tok0 + tl) * e.gate_stride + gcol]));
+            const int64_t off = row * e.row_stride + colpart;
+            if (e.out_f32)
+              static_cast<float*>(e.out)[off] = val;
+            else
+              static_cast<__nv_bfloat16*>(e.out)[off] = __float2bfloat16_rn(val);
+          }
+        };
+        if (a.splits <= 1) {
+#pragma unroll 1
+          for (int c0 = 0; c0 < BN; c0 += 16) {
+            uint32_t v[16];
+            tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + c0, v);
+            tmem_ld_wait();
+            float x[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) x[j] = __uint_as_float(v[j]);
+            if (acc_ok) store_chunk(c0, x);
+          }
+        } else {
+          // publish this split's partial (row-major: each thread writes its own
+          // row), take a ticket, and let the last split sum and store
+          const int tiles = gridDim.x * gridDim.y;
+          const int tile_id = blockIdx.y * gridDim.x + blockIdx.x;
+          float* mine = a.partial + (static_cast<size_t>(blockIdx.z) * tiles + tile_id) * (128 * BN) + r * BN;
+#pragma unroll 1
+          for (int c0 = 0; c0 < BN; c0 += 16) {
+            uint32_t v[16];
+            tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + c0, v);
+            tmem_ld_wait();
+            if (acc_ok) {
+#pragma unroll
+              for (int j = 0; j < 16; j += 4)
+                *reinterpret_cast<float4*>(mine + c0 + j) =
+                    make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]), __uint_as_float(v[j + 2]),
+                                __uint_as_float(v[j + 3]));
+            }
+          }
+          __threadfence();
+          asm volatile("bar.sync 2, 128;" ::: "memory");
+          if (threadIdx.x == 64) *last_flag = (atomicAdd(&a.counters[tile_id], 1) == a.splits - 1) ? 1 : 0;
+          asm volatile("bar.sync 2, 128;" ::: "memory");
+          if (*last_flag && acc_ok) {
+            __threadfence();
+#pragma unroll 1
+            for (int c0 = 0; c0 < BN; c0 += 16) {
+              float x[16];
+#pragma unroll
+              for (int j = 0; j < 16; ++j) x[j] = 0.f;
+              // issue the loads of up to 8 splits before summing any of them
+#pragma unroll 1
+              for (int z0 = 0; z0 < a.splits; z0 += 8) {
+                float4 u[8][4];
+#pragma unroll
+                for (int z = 0; z < 8; ++z) {
+                  if (z0 + z < a.splits) {
+                    const float4* pz = reinterpret_cast<const float4*>(
+                        a.partial + (static_cast<size_t>(z0 + z) * tiles + tile_id) * (128 * BN) + r * BN + c0);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) u[z][j] = __ldcg(pz + j);
+                  } else {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) u[z][j] = make_float4(0.f, 0.f, 0.f, 0.f);
+                  }
+                }
+#pragma unroll
+                for (int z = 0; z < 8; ++z)
+#pragma unroll
+                  for (int j = 0; j < 4; ++j) {
+                    x[4 * j] += u[z][j].x;
+                    x[4 * j + 1] += u[z][j].y;
+                    x[4 * j + 2] += u[z][j].z;
+                    x[4 * j + 3] += u[z][j].w;
+                  }
               }
+              store_chunk(c0, x);
             }
-            epi_store(e, row, f, val);
+            if (threadIdx.x == 64) a.counters[tile_id] = 0;
           }
         }
       } else {
@@ -229,7 +335,7 @@ __global__ void __launch_bounds__(192, 1) gemm_bf16_tc_kernel(const __grid_const
               x[j + 1] = rope_rotate(x1, x0, true, pos, fi >> 1, e.block, a.log2_rope_base);
             }
           }
-          const bool vec = !e.out_f32 && !e.bias && (f0 + 16 <= seg_rows) && (f0 % e.block) + 16 <= e.block &&
+          const bool vec = !e.out_f32 && !e.bias && !e.gate && (f0 + 16 <= seg_rows) && (f0 % e.block) + 16 <= e.block &&
                            ((row * e.row_stride + (f0 / e.block) * (int64_t)e.block_stride + (f0 % e.block) +
                              e.col_offset) % 8 == 0);
           if (vec) {
@@ -250,7 +356,7 @@ __global__ void __launch_bounds__(192, 1) gemm_bf16_tc_kernel(const __grid_const
           } else {
 #pragma unroll
             for (int j = 0; j < 16; ++j)
-              if (f0 + j < seg_rows) epi_store(e, row, f0 + j, x[j]);
+              if (f0 + j < seg_rows) epi_store(e, row, f0 + j, x[j], tok);
           }
         }
       }
@@ -279,8 +385,33 @@ static cudaError_t launch_one(const GemmArgs& a, dim3 grid, cudaStream_t st) {
 
 int gemm_weight_tile(bool swap, int bn) { return swap ? 128 : bn; }
 
+int gemm_swap_bn(int T) { return T <= 16 ? 16 : T <= 32 ? 32 : T <= 64 ? 64 : T <= 128 ? 128 : 256; }
+
+SwapPlan gemm_swap_plan(int wtiles, int T, int K, int num_sms) {
+  SwapPlan p{};
+  p.bn = gemm_swap_bn(T);
+  p.ttiles = (T + p.bn - 1) / p.bn;
+  const int tiles = wtiles * p.ttiles;
+  const int num_kb = (K + 63) / 64;
+  // Two CTAs fit on an SM. Few tiles: split K until the tiles fill one wave.
+  // Many tiles: split so there are at least four waves (tail imbalance < 25%).
+  const int slots = 2 * num_sms;
+  int splits = 1;
+  if (tiles > 0) splits = tiles <= slots ? slots / tiles : (4 * slots + tiles - 1) / tiles;
+  const int max_splits = num_kb / 4 > 1 ? num_kb / 4 : 1;   // keep >= 4 K blocks per split
+  splits = splits < 1 ? 1 : (splits > max_splits ? max_splits : splits);
+  if (splits > 16) splits = 16;
+  p.kb_per_split = (num_kb + splits - 1) / splits;
+  p.splits = (num_kb + p.kb_per_split - 1) / p.kb_per_split;
+  p.tiles = tiles;
+  p.ws_bytes = p.splits > 1 ? (static_cast<size_t>(tiles) * 4 + 255) / 256 * 256 +
+                                  static_cast<size_t>(p.splits) * tiles * 128 * p.bn * 4
+                            : 0;
+  return p;
+}
+
 cudaError_t launch_gemm_bf16(const GemmArgs& a, bool swap, int bn, int token_tiles, cudaStream_t st) {
-  dim3 grid(a.seg_tile_begin[a.n_seg], token_tiles);
+  dim3 grid(a.seg_tile_begin[a.n_seg], token_tiles, swap ? (a.splits > 1 ? a.splits : 1) : 1);
   if (grid.x == 0 || grid.y == 0) return cudaSuccess;
   if (swap) {
     switch (bn) {

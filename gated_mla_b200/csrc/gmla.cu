@@ -172,6 +172,16 @@ size_t g_prof_used = 0;
 bool g_prof_open = false;
 std::atomic<uint64_t> g_launches{0};
 
+// Point a swap-orientation GEMM at its split-K scratch and zero the tickets.
+cudaError_t set_splits(GemmArgs& a, const SwapPlan& sp, uint8_t* ws, cudaStream_t st) {
+  a.splits = sp.splits;
+  a.kb_per_split = sp.kb_per_split;
+  if (sp.splits <= 1) return cudaSuccess;
+  a.counters = reinterpret_cast<int32_t*>(ws);
+  a.partial = reinterpret_cast<float*>(ws + align256(static_cast<size_t>(sp.tiles) * 4));
+  return cudaMemsetAsync(ws, 0, static_cast<size_t>(sp.tiles) * 4, st);
+}
+
 }  // namespace
 
 namespace gmla {
@@ -268,22 +278,32 @@ gmla_status gmla_profile_get(int32_t i, const char** name, float* ms) {
   return GMLA_OK;
 }
 
+static int project_wtiles(const gmla_config* c) {
+  const int G = c->gate_mode == GMLA_GATE_CHANNEL ? c->n_heads * c->d_h : c->n_heads;
+  const int rows[5] = {c->d_c, c->d_rope, c->n_heads * c->d_h, c->n_heads * c->d_rope, G};
+  int t = 0;
+  for (int r : rows) t += (r + 127) / 128;
+  return t;
+}
+
 size_t gmla_latent_project_workspace_size(const gmla_config* cfg, int32_t T) {
-  (void)cfg;
-  (void)T;
-  return 256;
+  if (!cfg || T < 0 || cfg->dtype == GMLA_FP32 || T > 256) return 256;
+  return 256 + gemm_swap_plan(project_wtiles(cfg), T, cfg->d_model, num_sms()).ws_bytes;
 }
 
 size_t gmla_gate_out_workspace_size(const gmla_config* cfg, int32_t T) {
   if (!cfg || T < 0) return 256;
   const size_t es = cfg->dtype == GMLA_FP32 ? 4 : 2;
-  return 256 + align256(static_cast<size_t>(T) * cfg->n_heads * cfg->d_h * es);
+  size_t n = 256 + align256(static_cast<size_t>(T) * cfg->n_heads * cfg->d_h * es);
+  if (cfg->dtype != GMLA_FP32 && T <= 256)
+    n += gemm_swap_plan((cfg->d_model + 127) / 128, T, cfg->n_heads * cfg->d_h, num_sms()).ws_bytes;
+  return n;
 }
 
 size_t gmla_decode_workspace_size(const gmla_config* cfg, int32_t B) {
   if (!cfg || B < 0) return 256;
   if (cfg->dtype == GMLA_FP32) return 256;
-  return decode_layout(B, cfg->n_heads, cfg->d_c, cfg->d_rope, num_sms()).total;
+  return decode_layout(B, cfg->n_heads, cfg->d_h, cfg->d_c, cfg->d_rope, num_sms()).total;
 }
 
 size_t gmla_prefill_workspace_size(const gmla_config* cfg, int32_t T, int32_t B) {
@@ -383,7 +403,8 @@ gmla_status gmla_latent_project(const gmla_config* cfg, const gmla_weights* w, c
   if (dm % 8) return fail(GMLA_ERR_UNSUPPORTED, "bf16 path needs d_model %% 8 == 0");
   GemmArgs a{};
   const bool swap = T <= 256;
-  const int bn = swap ? (T <= 16 ? 16 : T <= 32 ? 32 : T <= 64 ? 64 : T <= 128 ? 128 : 256) : 256;
+  const SwapPlan sp = gemm_swap_plan(project_wtiles(cfg), T, dm, num_sms());
+  const int bn = swap ? sp.bn : 256;
   const int wtile = gemm_weight_tile(swap, bn);
   if (!make_tmap_2d(&a.act, x, dm, T, static_cast<uint64_t>(dm) * 2, 64, swap ? bn : 128, true))
     return fail(GMLA_ERR_CUDA, "tensor map for x failed");
@@ -404,8 +425,10 @@ gmla_status gmla_latent_project(const gmla_config* cfg, const gmla_weights* w, c
   a.cache = cv;
   a.log2_rope_base = dr ? std::log2(static_cast<double>(cfg->rope_base)) : 0.0;
   a.status = status;
-  const int ttiles = swap ? (T + bn - 1) / bn : (T + 127) / 128;
-  cudaError_t e = launch_gemm_bf16(a, swap, bn, ttiles, st);
+  const int ttiles = swap ? sp.ttiles : (T + 127) / 128;
+  cudaError_t e = cudaSuccess;
+  if (swap) e = set_splits(a, sp, static_cast<uint8_t*>(workspace) + 256, st);
+  if (e == cudaSuccess) e = launch_gemm_bf16(a, swap, bn, ttiles, st);
   return e == cudaSuccess ? GMLA_OK : cuda_fail(e, "latent_project");
 }
 
@@ -459,19 +482,20 @@ gmla_status gmla_decode(const gmla_config* cfg, const gmla_weights* w, const voi
 
   if (cfg->d_c != 512 || (cfg->d_rope != 0 && cfg->d_rope != 64))
     return fail(GMLA_ERR_UNSUPPORTED, "bf16 decode covers d_c = 512 with d_rope in {0, 64}");
-  if (cfg->d_h % 4 || cfg->d_h > 256) return fail(GMLA_ERR_UNSUPPORTED, "bf16 decode needs d_h %% 4 == 0, <= 256");
-  const DecodeLayout L = decode_layout(B, cfg->n_heads, cfg->d_c, cfg->d_rope, num_sms());
+  if (cfg->d_h != 128 && cfg->d_h != 256) return fail(GMLA_ERR_UNSUPPORTED, "bf16 decode covers d_h in {128, 256}");
+  const DecodeLayout L = decode_layout(B, cfg->n_heads, cfg->d_h, cfg->d_c, cfg->d_rope, num_sms());
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   DecodeArgs a{};
   const int row = cfg->d_c + cfg->d_rope;
+  const int tile_rows = 128;   // tokens per attention tile
   if (!cache->paged) {
     if (!make_tmap_2d(&a.cache_map, cache->data, row, static_cast<uint64_t>(cache->batch) * cache->capacity,
-                      static_cast<uint64_t>(row) * 2, 64, 128, true))
+                      static_cast<uint64_t>(row) * 2, 64, tile_rows, true))
       return fail(GMLA_ERR_CUDA, "tensor map for the cache failed");
   } else {
     const int ps = cache->page_size;
     if (!make_tmap_3d(&a.cache_map, cache->data, row, ps, cache->num_pages, static_cast<uint64_t>(row) * 2,
-                      static_cast<uint64_t>(row) * 2 * ps, 64, ps < 128 ? ps : 128, 1, true))
+                      static_cast<uint64_t>(row) * 2 * ps, 64, ps < tile_rows ? ps : tile_rows, 1, true))
       return fail(GMLA_ERR_CUDA, "tensor map for the paged cache failed");
   }
   if (!make_tmap_2d(&a.qa_map, ws + L.off_qa, row, static_cast<uint64_t>(B) * cfg->n_heads,
@@ -502,7 +526,40 @@ gmla_status gmla_decode(const gmla_config* cfg, const gmla_weights* w, const voi
   a.G = L.G;
   a.max_seg = L.max_seg;
   a.q_scale = cfg->softmax_scale * 1.4426950408889634f;
+  a.olat = ws + L.off_olat;
+  const SwapPlan& sp = L.gemm_plan;
+  a.gemm_counters = reinterpret_cast<int32_t*>(ws + L.off_gemm);
+  a.n_gemm_tiles = sp.splits > 1 ? sp.tiles : 0;
+
+  // o = sigmoid(g) ⊙ W_v^(h) O_lat^(h): a swap-orientation GEMM over heads
+  const int HD = cfg->n_heads * cfg->d_h;
+  const int G = gate_width(cfg);
+  GemmArgs g{};
+  if (!make_tmap_2d(&g.act, a.olat, cfg->d_c, static_cast<uint64_t>(cfg->n_heads) * B,
+                    static_cast<uint64_t>(cfg->d_c) * 2, 64, sp.bn, true) ||
+      !make_tmap_2d(&g.wt[0], w->W_v, cfg->d_c, HD, static_cast<uint64_t>(cfg->d_c) * 2, 64, 128, true))
+    return fail(GMLA_ERR_CUDA, "tensor maps for the W_v product failed");
+  g.epi[0] = plain_seg(o_gated, HD, 1 << 30, 0, 0, false, nullptr, false, false);
+  g.epi[0].gate = gate_logits;
+  g.epi[0].gate_stride = G;
+  g.epi[0].gate_div = cfg->gate_mode == GMLA_GATE_CHANNEL ? 1 : cfg->d_h;
+  g.seg_rows[0] = HD;
+  g.seg_tile_begin[0] = 0;
+  g.seg_tile_begin[1] = HD / 128;
+  g.n_seg = 1;
+  g.T = B;
+  g.K = cfg->d_c;
+  g.row_mode = 2;
+  g.rows_per_group = cfg->d_h;
+  g.act_group_stride = B;
+  g.splits = sp.splits;
+  g.kb_per_split = sp.kb_per_split;
+  g.counters = a.gemm_counters;
+  g.partial = reinterpret_cast<float*>(ws + L.off_gemm + align256(static_cast<size_t>(sp.tiles) * 4));
+  g.status = status;
+
   cudaError_t e = launch_decode_bf16(a, st);
+  if (e == cudaSuccess) e = launch_gemm_bf16(g, true, sp.bn, sp.ttiles, st);
   return e == cudaSuccess ? GMLA_OK : cuda_fail(e, "decode");
 }
 
@@ -660,7 +717,8 @@ gmla_status gmla_gate_out(const gmla_config* cfg, const gmla_weights* w, const v
   if (HD % 8) return fail(GMLA_ERR_UNSUPPORTED, "bf16 path needs H*d_h %% 8 == 0");
   GemmArgs a{};
   const bool swap = T <= 256;
-  const int bn = swap ? (T <= 16 ? 16 : T <= 32 ? 32 : T <= 64 ? 64 : T <= 128 ? 128 : 256) : 256;
+  const SwapPlan sp = gemm_swap_plan((dm + 127) / 128, T, HD, num_sms());
+  const int bn = swap ? sp.bn : 256;
   const int wtile = gemm_weight_tile(swap, bn);
   if (!make_tmap_2d(&a.act, src, HD, T, static_cast<uint64_t>(HD) * 2, 64, swap ? bn : 128, true) ||
       !make_tmap_2d(&a.wt[0], w->W_o, HD, dm, static_cast<uint64_t>(HD) * 2, 64, wtile, true))
@@ -674,8 +732,10 @@ gmla_status gmla_gate_out(const gmla_config* cfg, const gmla_weights* w, const v
   a.K = HD;
   a.row_mode = 0;
   a.status = status;
-  const int ttiles = swap ? (T + bn - 1) / bn : (T + 127) / 128;
-  cudaError_t e = launch_gemm_bf16(a, swap, bn, ttiles, st);
+  const int ttiles = swap ? sp.ttiles : (T + 127) / 128;
+  cudaError_t e = cudaSuccess;
+  if (swap) e = set_splits(a, sp, static_cast<uint8_t*>(workspace) + 256 + align256(static_cast<size_t>(T) * HD * 2), st);
+  if (e == cudaSuccess) e = launch_gemm_bf16(a, swap, bn, ttiles, st);
   return e == cudaSuccess ? GMLA_OK : cuda_fail(e, "gate_out");
 }
 

@@ -12,6 +12,14 @@ namespace gmla {
 // ----- tcgen05 GEMM (gemm_tc.cu) -----
 cudaError_t launch_gemm_bf16(const GemmArgs& a, bool swap, int bn, int token_tiles, cudaStream_t st);
 int gemm_weight_tile(bool swap, int bn);
+int gemm_swap_bn(int T);
+// Tiling of the swap orientation (few tokens): token tile width, K splits and
+// the workspace they need (ticket counters, then fp32 partial tiles).
+struct SwapPlan {
+  int bn, ttiles, tiles, splits, kb_per_split;
+  size_t ws_bytes;
+};
+SwapPlan gemm_swap_plan(int wtiles, int T, int K, int num_sms);
 
 // ----- decode (decode_tc.cu) -----
 struct DecodeArgs {
@@ -30,6 +38,9 @@ struct DecodeArgs {
   int4* seg_info;            // workspace: [max_seg]
   int32_t* seq_first_seg;    // workspace: [B + 1]
   int32_t* cta_first_seg;    // workspace: [G + 1]
+  void* olat;                // workspace: [H, B, d_c] bf16 merged latent outputs
+  int32_t* gemm_counters;    // workspace: split-K tickets of the W_v GEMM
+  int32_t n_gemm_tiles;
   int* status;
   int32_t B, H, d_h, d_c, d_rope, gate_mode;
   int32_t HG, n_hg, G, max_seg;
@@ -37,10 +48,11 @@ struct DecodeArgs {
 };
 
 struct DecodeLayout {
-  size_t off_qa, off_opart, off_ml, off_seg, off_seqfirst, off_ctafirst, total;
+  size_t off_qa, off_opart, off_ml, off_seg, off_seqfirst, off_ctafirst, off_olat, off_gemm, total;
   int HG, n_hg, G, max_seg;
+  SwapPlan gemm_plan;        // the W_v GEMM (heads x 128 rows, B tokens, K = d_c)
 };
-DecodeLayout decode_layout(int B, int H, int d_c, int d_rope, int num_sms);
+DecodeLayout decode_layout(int B, int H, int d_h, int d_c, int d_rope, int num_sms);
 cudaError_t launch_decode_bf16(DecodeArgs& a, cudaStream_t st);
 
 // ----- fp32 CUDA-core path (simt_f32.cu) -----
