@@ -77,12 +77,10 @@ struct GemmArgs {
   //   sequence * act_seq_stride, packed tokens at cu_seqlens[sequence].
   int32_t row_mode;
   // split-K (swap orientation only): blockIdx.z is the split; each split
-  // accumulates kb_per_split 64-wide K blocks, writes an fp32 partial tile and
-  // the last split to finish (ticket in counters[tile]) sums and stores.
+  // accumulates kb_per_split 64-wide K blocks; the splits of a tile run as one
+  // cluster and rank 0 sums their partials through distributed shared memory.
   int32_t splits;
   int32_t kb_per_split;
-  float* partial;            // [splits][tiles][BN][128] fp32
-  int32_t* counters;         // [tiles], zero before the launch
   int32_t tiles_per_seq;
   int32_t act_seq_stride;
   const int32_t* cu_seqlens;

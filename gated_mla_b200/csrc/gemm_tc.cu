@@ -80,7 +80,6 @@ __global__ void __launch_bounds__(192, 1) gemm_bf16_tc_kernel(const __grid_const
   uint64_t* drain = acc_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  volatile int* last_flag = abort_flag + 1;
   // per-token output row and position of this tile (swap orientation), filled once
   int64_t* tok_row = reinterpret_cast<int64_t*>(smem + C::kStages * C::kStageBytes + 256);
   int* tok_pos = reinterpret_cast<int*>(tok_row + (kSwap ? BN : 1));
@@ -245,64 +244,22 @@ __global__ void __launch_bounds__(192, 1) gemm_bf16_tc_kernel(const __grid_const
             if (acc_ok) store_chunk(c0, x);
           }
         } else {
-          // publish this split's partial (row-major: each thread writes its own
-          // row), take a ticket, and let the last split sum and store
-          const int tiles = gridDim.x * gridDim.y;
-          const int tile_id = blockIdx.y * gridDim.x + blockIdx.x;
-          float* mine = a.partial + (static_cast<size_t>(blockIdx.z) * tiles + tile_id) * (128 * BN) + r * BN;
+          // K splits of this tile form one cluster: every split leaves its fp32
+          // partial in its own (now idle) stage memory, rank 0 sums them over
+          // distributed shared memory and stores. Both cluster barriers are
+          // reached on every path so no CTA waits for one that left.
+          float* part = reinterpret_cast<float*>(smem) + r * (BN + 4);   // [128][BN + 4]
 #pragma unroll 1
           for (int c0 = 0; c0 < BN; c0 += 16) {
             uint32_t v[16];
             tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + c0, v);
             tmem_ld_wait();
-            if (acc_ok) {
 #pragma unroll
-              for (int j = 0; j < 16; j += 4)
-                *reinterpret_cast<float4*>(mine + c0 + j) =
-                    make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]), __uint_as_float(v[j + 2]),
-                                __uint_as_float(v[j + 3]));
-            }
-          }
-          __threadfence();
-          asm volatile("bar.sync 2, 128;" ::: "memory");
-          if (threadIdx.x == 64) *last_flag = (atomicAdd(&a.counters[tile_id], 1) == a.splits - 1) ? 1 : 0;
-          asm volatile("bar.sync 2, 128;" ::: "memory");
-          if (*last_flag && acc_ok) {
-            __threadfence();
-#pragma unroll 1
-            for (int c0 = 0; c0 < BN; c0 += 16) {
-              float x[16];
-#pragma unroll
-              for (int j = 0; j < 16; ++j) x[j] = 0.f;
-              // issue the loads of up to 8 splits before summing any of them
-#pragma unroll 1
-              for (int z0 = 0; z0 < a.splits; z0 += 8) {
-                float4 u[8][4];
-#pragma unroll
-                for (int z = 0; z < 8; ++z) {
-                  if (z0 + z < a.splits) {
-                    const float4* pz = reinterpret_cast<const float4*>(
-                        a.partial + (static_cast<size_t>(z0 + z) * tiles + tile_id) * (128 * BN) + r * BN + c0);
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) u[z][j] = __ldcg(pz + j);
-                  } else {
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) u[z][j] = make_float4(0.f, 0.f, 0.f, 0.f);
-                  }
-                }
-#pragma unroll
-                for (int z = 0; z < 8; ++z)
-#pragma unroll
-                  for (int j = 0; j < 4; ++j) {
-                    x[4 * j] += u[z][j].x;
-                    x[4 * j + 1] += u[z][j].y;
-                    x[4 * j + 2] += u[z][j].z;
-                    x[4 * j + 3] += u[z][j].w;
-                  }
-              }
-              store_chunk(c0, x);
-            }
-            if (threadIdx.x == 64) a.counters[tile_id] = 0;
+            for (int j = 0; j < 16; j += 4)
+              *reinterpret_cast<float4*>(part + c0 + j) =
+                  acc_ok ? make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]), __uint_as_float(v[j + 2]),
+                                       __uint_as_float(v[j + 3]))
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
           }
         }
       } else {
@@ -363,6 +320,61 @@ __global__ void __launch_bounds__(192, 1) gemm_bf16_tc_kernel(const __grid_const
     }
   }
 
+  if (kSwap && a.splits > 1) {
+    cluster_sync_all();   // every split's partial is in its shared memory
+    // reduce-scatter: rank z sums columns [z*cpr, (z+1)*cpr) of every split's
+    // partial (one float4 per split per row, all loads in flight together)
+    // and stores them
+    const int cpr = ((BN + a.splits - 1) / a.splits + 3) & ~3;
+    const int col0 = static_cast<int>(cluster_ctarank()) * cpr;
+    if (warp >= 2 && col0 < BN) {
+      const int q = warp & 3, r = q * 32 + lane;
+      const int f = tile.wrow0 + r;
+      const EpiSeg e = a.epi[tile.seg];
+      const int seg_rows = a.seg_rows[tile.seg];
+      const bool f_ok = f < seg_rows;
+      const int64_t colpart = static_cast<int64_t>(f / e.block) * e.block_stride + (f % e.block) + e.col_offset;
+      const float fbias = (e.bias && f_ok) ? e.bias[f] : 0.f;
+      const int gcol = e.gate ? f / e.gate_div : 0;
+      const uint32_t part = smem_u32(smem) + r * (BN + 4) * 4;
+#pragma unroll 1
+      for (int c0 = col0; c0 < min(BN, col0 + cpr); c0 += 4) {
+        float4 u[8];
+#pragma unroll
+        for (int z = 0; z < 8; ++z)
+          u[z] = z < a.splits ? ld_cluster_f4(cluster_map(part, z) + c0 * 4) : make_float4(0.f, 0.f, 0.f, 0.f);
+        float x[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int z = 0; z < 8; ++z) {
+          x[0] += u[z].x;
+          x[1] += u[z].y;
+          x[2] += u[z].z;
+          x[3] += u[z].w;
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int tl = c0 + j;
+          float val = x[j];
+          if (e.rope) {
+            const float partner = __shfl_xor_sync(0xffffffffu, val, 1);
+            const int fi = f % e.block;
+            val = rope_rotate(val, partner, fi & 1, tok_pos[tl], fi >> 1, e.block, a.log2_rope_base);
+          }
+          const int64_t row = tok_row[tl];
+          if (row < 0 || !f_ok || *abort_flag) continue;
+          val += fbias;
+          if (e.gate) val *= 1.f / (1.f + __expf(-e.gate[static_cast<int64_t>(tile.tok0 + tl) * e.gate_stride + gcol]));
+          const int64_t off = row * e.row_stride + colpart;
+          if (e.out_f32)
+            static_cast<float*>(e.out)[off] = val;
+          else
+            static_cast<__nv_bfloat16*>(e.out)[off] = __float2bfloat16_rn(val);
+        }
+      }
+    }
+    cluster_sync_all();   // rank 0 has finished reading the other splits' memory
+  }
+
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -378,9 +390,27 @@ static cudaError_t launch_one(const GemmArgs& a, dim3 grid, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   prof_begin(st, kSwap ? "gemm_bf16_swap" : "gemm_bf16");
-  k<<<grid, 192, C::kSmemBytes, st>>>(a);
+  if (kSwap && a.splits > 1) {
+    // the K splits of one tile run as a cluster along z
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(192);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = a.splits;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, k, a);
+  } else {
+    k<<<grid, 192, C::kSmemBytes, st>>>(a);
+    e = cudaGetLastError();
+  }
   prof_end(st);
-  return cudaGetLastError();
+  return e;
 }
 
 int gemm_weight_tile(bool swap, int bn) { return swap ? 128 : bn; }
@@ -393,20 +423,19 @@ SwapPlan gemm_swap_plan(int wtiles, int T, int K, int num_sms) {
   p.ttiles = (T + p.bn - 1) / p.bn;
   const int tiles = wtiles * p.ttiles;
   const int num_kb = (K + 63) / 64;
-  // Two CTAs fit on an SM. Few tiles: split K until the tiles fill one wave.
-  // Many tiles: split so there are at least four waves (tail imbalance < 25%).
-  const int slots = 2 * num_sms;
+  // Few tiles: split K (one cluster of splits per tile) until the tiles fill one
+  // CTA per SM. Many tiles: split so there are at least four waves of two CTAs
+  // per SM (tail imbalance < 25%).
+  const int slots = tiles <= num_sms ? num_sms : 2 * num_sms;
   int splits = 1;
   if (tiles > 0) splits = tiles <= slots ? slots / tiles : (4 * slots + tiles - 1) / tiles;
   const int max_splits = num_kb / 4 > 1 ? num_kb / 4 : 1;   // keep >= 4 K blocks per split
   splits = splits < 1 ? 1 : (splits > max_splits ? max_splits : splits);
-  if (splits > 16) splits = 16;
+  if (splits > 8) splits = 8;   // the splits of a tile form one (portable-size) cluster
   p.kb_per_split = (num_kb + splits - 1) / splits;
   p.splits = (num_kb + p.kb_per_split - 1) / p.kb_per_split;
   p.tiles = tiles;
-  p.ws_bytes = p.splits > 1 ? (static_cast<size_t>(tiles) * 4 + 255) / 256 * 256 +
-                                  static_cast<size_t>(p.splits) * tiles * 128 * p.bn * 4
-                            : 0;
+  p.ws_bytes = 0;               // partials are reduced through distributed shared memory
   return p;
 }
 

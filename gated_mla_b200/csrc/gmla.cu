@@ -172,14 +172,13 @@ size_t g_prof_used = 0;
 bool g_prof_open = false;
 std::atomic<uint64_t> g_launches{0};
 
-// Point a swap-orientation GEMM at its split-K scratch and zero the tickets.
+// K split of a swap-orientation GEMM (the splits reduce through a cluster).
 cudaError_t set_splits(GemmArgs& a, const SwapPlan& sp, uint8_t* ws, cudaStream_t st) {
+  (void)ws;
+  (void)st;
   a.splits = sp.splits;
   a.kb_per_split = sp.kb_per_split;
-  if (sp.splits <= 1) return cudaSuccess;
-  a.counters = reinterpret_cast<int32_t*>(ws);
-  a.partial = reinterpret_cast<float*>(ws + align256(static_cast<size_t>(sp.tiles) * 4));
-  return cudaMemsetAsync(ws, 0, static_cast<size_t>(sp.tiles) * 4, st);
+  return cudaSuccess;
 }
 
 }  // namespace
@@ -198,7 +197,7 @@ void prof_begin(cudaStream_t st, const char* name) {
     g_prof.push_back(r);
   }
   g_prof[g_prof_used].name = name;
-  cudaEventRecord(g_prof[g_prof_used].start, st);
+  cudaEventRecordWithFlags(g_prof[g_prof_used].start, st, cudaEventRecordExternal);
   g_prof_open = true;
 }
 
@@ -206,7 +205,7 @@ void prof_end(cudaStream_t st) {
   if (!g_prof_on) return;
   std::lock_guard<std::mutex> lk(g_prof_mu);
   if (!g_prof_open) return;
-  cudaEventRecord(g_prof[g_prof_used].stop, st);
+  cudaEventRecordWithFlags(g_prof[g_prof_used].stop, st, cudaEventRecordExternal);
   ++g_prof_used;
   g_prof_open = false;
 }
@@ -528,8 +527,8 @@ gmla_status gmla_decode(const gmla_config* cfg, const gmla_weights* w, const voi
   a.q_scale = cfg->softmax_scale * 1.4426950408889634f;
   a.olat = ws + L.off_olat;
   const SwapPlan& sp = L.gemm_plan;
-  a.gemm_counters = reinterpret_cast<int32_t*>(ws + L.off_gemm);
-  a.n_gemm_tiles = sp.splits > 1 ? sp.tiles : 0;
+  a.gemm_counters = nullptr;
+  a.n_gemm_tiles = 0;
 
   // o = sigmoid(g) ⊙ W_v^(h) O_lat^(h): a swap-orientation GEMM over heads
   const int HD = cfg->n_heads * cfg->d_h;
@@ -554,8 +553,6 @@ gmla_status gmla_decode(const gmla_config* cfg, const gmla_weights* w, const voi
   g.act_group_stride = B;
   g.splits = sp.splits;
   g.kb_per_split = sp.kb_per_split;
-  g.counters = a.gemm_counters;
-  g.partial = reinterpret_cast<float*>(ws + L.off_gemm + align256(static_cast<size_t>(sp.tiles) * 4));
   g.status = status;
 
   cudaError_t e = launch_decode_bf16(a, st);
