@@ -1,14 +1,18 @@
 #!/usr/bin/env python
-"""Benchmark of the Gated MLA decode hot path on B200.
+"""Benchmark of the Gated MLA hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME]
 
-A step is one pass of the whole decode path over the batch-32 decode workload
-(d_model 2048, 16 heads, d_h 128, d_c 512, NoPE, per-channel gate, cache
-lengths uniform in [1024, 8192], seed 0): gmla_latent_project (writes each
-sequence's new latent row) -> gmla_decode (absorbed split-K attention, W_v
-and gate) -> gmla_gate_out (W_o). The metric is latent-cache bytes read per
-step over the step time (GB/s). Inputs are synthetic, drawn by ``synth``.
+Default workload: the batch-32 decode (d_model 2048, 16 heads, d_h 128,
+d_c 512, NoPE, per-channel gate, cache lengths uniform in [1024, 8192],
+seed 0). A decode step is gmla_latent_project (writes each sequence's new
+latent row) -> gmla_decode (absorbed split-K attention, W_v and gate) ->
+gmla_gate_out (W_o); its metric is latent-cache bytes read per step over the
+step time (GB/s). A prefill step (``--workload prefill_b4_s4096`` or
+``tiny_prefill_f32``) is gmla_latent_project -> gmla_prefill -> gmla_gate_out
+over whole prompts; its metric is explicit-form algorithmic FLOPs per second
+(TFLOP/s). Inputs are synthetic, drawn by ``synth``.
 
 Timing: W untimed warm-up steps; then K steps, each replayed from a CUDA
 graph between CUDA events on the launching stream, with a 256 MiB memset
@@ -36,9 +40,9 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-METRIC = "Gated-MLA decode latent-cache GB/s (latent_project + decode + gate_out step)"
-UNIT = "GB/s"
-WORKLOAD = "decode_b32"
+DECODE_METRIC = "Gated-MLA decode latent-cache GB/s (latent_project + decode + gate_out step)"
+PREFILL_METRIC = "Gated-MLA prefill TFLOP/s (latent_project + prefill + gate_out step, explicit-form FLOPs)"
+DEFAULT_WORKLOAD = "decode_b32"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 
 
@@ -48,6 +52,9 @@ def parse():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                    choices=["decode_b32", "decode_long_rope", "decode_paged_head", "prefill_b4_s4096",
+                             "tiny_prefill_f32"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle CPU baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
@@ -144,6 +151,40 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------
+# workload accounting
+# ---------------------------------------------------------------------------
+
+def prefill_flops(w, lengths):
+    """Explicit-form algorithmic FLOPs of one prefill step, per kernel."""
+    T = int(sum(lengths))
+    H, dh, dc, dr, dm = w.n_heads, w.d_h, w.d_c, w.d_rope, w.d_model
+    n_proj = dc + dr + H * dh + H * dr + w.gate_width
+    pairs = sum(int(L) * (int(L) + 1) // 2 for L in lengths)
+    return {"gemm_project": 2.0 * T * dm * n_proj,
+            "gemm_kv": 2.0 * T * dc * 2 * H * dh,
+            "prefill_attn": 4.0 * (dh + dr) * H * pairs,
+            "gemm_out": 2.0 * T * H * dh * dm}
+
+
+def config_dict(w, inp):
+    lens = inp["lengths"]
+    if w.mode == "decode":
+        desc = (f"{w.name}: batch {w.batch} decode, d_model {w.d_model}, H {w.n_heads}, d_h {w.d_h}, d_c {w.d_c}"
+                + (f" + RoPE {w.d_rope}" if w.d_rope else ", NoPE")
+                + (", paged (page 64)" if w.paged else "")
+                + f", {w.gate_mode} gate, lengths {w.len_law}[{w.len_lo},{w.len_hi}] seed 0")
+        extra = {"sum_len": int(lens.sum()), "latent_bytes_per_step": int(lens.sum()) * w.row * 2}
+    else:
+        desc = (f"{w.name}: batch {w.batch} x {w.seq_len} causal prefill, d_model {w.d_model}, H {w.n_heads}, "
+                f"d_h {w.d_h}, d_c {w.d_c}, NoPE, {w.gate_mode} gate, {w.dtype}")
+        extra = {"flops_per_step": sum(prefill_flops(w, lens).values())}
+    return dict({"workload": desc, "batch": w.batch, "d_model": w.d_model, "n_heads": w.n_heads, "d_h": w.d_h,
+                 "d_c": w.d_c, "d_rope": w.d_rope,
+                 "l2": "flushed before every timed step (256 MiB memset, outside the events)",
+                 "parallelism": "replica per GPU"}, **extra)
+
+
+# ---------------------------------------------------------------------------
 # CPU oracle (baseline leg and reference arm)
 # ---------------------------------------------------------------------------
 
@@ -157,79 +198,166 @@ def blas_threads():
 
 
 def oracle_sample(inp, seconds: float, start: int = 0):
-    """Run the fp64 oracle's decode over whole sequences from `start` until the
-    time budget is spent. Returns (latent bytes processed, seconds, sequences)."""
+    """Run the fp64 oracle on a bounded sample of the workload. Decode: whole
+    sequences from `start` until the time budget is spent (work = latent bytes
+    read). Prefill: a prefix of sequence 0 (same dimensions, shorter prompt;
+    work = its algorithmic FLOPs). Returns (work, seconds, description)."""
     import oracle
     w = inp["workload"]
     p = oracle.params(inp)
-    row_bytes = w.row * 2
-    done, nbytes = [], 0
     t0 = time.perf_counter()
-    b = start
-    while True:
-        oracle.decode(p, inp["x"], inp["past"], seqs=[b % w.batch])
-        nbytes += int(inp["lengths"][b % w.batch]) * row_bytes
-        done.append(b % w.batch)
-        b += 1
-        if time.perf_counter() - t0 >= seconds or len(done) >= w.batch:
-            break
-    return nbytes, time.perf_counter() - t0, done
+    if w.mode == "decode":
+        # units of (sequence, 8 heads); work = that share of the sequence's latent bytes
+        units, nbytes, b = 0, 0.0, start
+        hc = min(8, w.n_heads)
+        while True:
+            seq = b % w.batch
+            for h0 in range(0, w.n_heads, hc):
+                heads = list(range(h0, min(w.n_heads, h0 + hc)))
+                oracle.decode(p, inp["x"], inp["past"], seqs=[seq], heads=heads)
+                nbytes += int(inp["lengths"][seq]) * w.row * 2 * len(heads) / w.n_heads
+                units += 1
+                if time.perf_counter() - t0 >= seconds:
+                    break
+            b += 1
+            if time.perf_counter() - t0 >= seconds or b - start >= w.batch:
+                break
+        return nbytes, time.perf_counter() - t0, f"{units} (sequence, {hc}-head) units from {b - start} sequences"
+    S = min(int(inp["lengths"][0]), 512)
+    oracle.prefill(p, inp["x"][:S], [S])
+    flops = sum(prefill_flops(w, [S]).values())
+    return flops, time.perf_counter() - t0, f"prefill of the first {S} tokens of sequence 0"
+
+
+def work_unit(w):
+    return (1e9, "GB/s") if w.mode == "decode" else (1e12, "TFLOP/s")
 
 
 def run_reference(args):
     import synth
     if int(os.environ.get("RANK", "0")) != 0:
         return
-    w = synth.workload(WORKLOAD)
+    w = synth.workload(args.workload)
     inp = synth.generate(w, seed=0)
+    scale, unit = work_unit(w)
     per_step = max(0.5, min(6.0, 150.0 / max(1, args.steps + args.warmup)))
     for i in range(args.warmup):
         oracle_sample(inp, per_step, start=i)
-    tot_b, tot_s, seqs = 0, 0.0, []
+    tot_w, tot_s, desc = 0.0, 0.0, ""
     for i in range(args.steps):
-        nb, s, d = oracle_sample(inp, per_step, start=args.warmup + i)
-        tot_b += nb
-        tot_s += s
-        seqs += d
-    value = tot_b / tot_s / 1e9
+        wk, sec, desc = oracle_sample(inp, per_step, start=args.warmup + i)
+        tot_w += wk
+        tot_s += sec
+    value = tot_w / tot_s / scale
     cores = blas_threads()
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_s / args.steps,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": config_dict(w, inp),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                         "sample": f"{len(seqs)} whole sequences over {args.steps} steps, fp64 explicit form "
-                                   f"(per-head K/V rebuilt from latents), numpy/BLAS"},
-        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "impl": "reference", "metric": DECODE_METRIC if w.mode == "decode" else PREFILL_METRIC,
+        "value": value, "unit": unit, "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * tot_s / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config_dict(w, inp),
+        "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle",
+                         "sample": f"per step: {desc}; fp64 explicit form (per-head K/V rebuilt from "
+                                   f"latents), numpy/BLAS"},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
-
-
-def config_dict(w, inp):
-    lens = inp["lengths"]
-    return {"workload": f"{WORKLOAD}: batch {w.batch} decode, d_model {w.d_model}, H {w.n_heads}, d_h {w.d_h}, "
-                        f"d_c {w.d_c}, NoPE, per-channel gate, lengths uniform[{w.len_lo},{w.len_hi}] seed 0",
-            "batch": w.batch, "d_model": w.d_model, "n_heads": w.n_heads, "d_h": w.d_h, "d_c": w.d_c,
-            "d_rope": w.d_rope, "sum_len": int(lens.sum()),
-            "latent_bytes_per_step": int(lens.sum()) * w.row * 2,
-            "l2": "flushed before every timed step (256 MiB memset, outside the events)",
-            "parallelism": "replica per GPU"}
 
 
 # ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
 
+class DecodeRunner:
+    def __init__(self, inp, dev):
+        import torch
+        sys.path.insert(0, os.path.join(ROOT, "tests"))
+        from gpu_pipeline import make_decode_cache, make_model
+        w = self.w = inp["workload"]
+        self.dev = dev
+        self.model = make_model(inp, device=dev)
+        self.cache = make_decode_cache(inp, device=dev, fill=0.0)
+        B = w.batch
+        self.x = torch.from_numpy(inp["x"]).to(dev, torch.bfloat16)
+        self.seq_lens = torch.tensor(inp["lengths"], dtype=torch.int32, device=dev)
+        self.positions = (self.seq_lens - 1).contiguous()
+        self.seq_ids = torch.arange(B, dtype=torch.int32, device=dev)
+        self.q = torch.empty(B, w.n_heads, w.d_h + w.d_rope, dtype=torch.bfloat16, device=dev)
+        self.g = torch.empty(B, w.gate_width, dtype=torch.float32, device=dev)
+        self.o = torch.empty(B, w.n_heads * w.d_h, dtype=torch.bfloat16, device=dev)
+        self.y = torch.empty(B, w.d_model, dtype=torch.bfloat16, device=dev)
+        self.work = float(inp["lengths"].sum()) * w.row * 2          # latent bytes per step
+        self.dominant = "decode_attn"
+        self.kernel_work = {"decode_attn": self.work}
+        # host copies for the end-to-end leg
+        self.host_in = [t.cpu().pin_memory() for t in (self.x, self.seq_lens, self.positions, self.seq_ids)]
+        self.dev_in = [torch.empty_like(t) for t in (self.x, self.seq_lens, self.positions, self.seq_ids)]
+        self.y_host = torch.empty(B, w.d_model, dtype=torch.bfloat16).pin_memory()
+
+    def step(self):
+        m = self.model
+        m.latent_project(self.x, self.positions, self.seq_ids, self.cache, q_out=self.q, gate_logits=self.g)
+        m.decode(self.q, self.g, self.cache, self.seq_lens, o_out=self.o)
+        m.gate_out(self.o, y_out=self.y)
+
+    def e2e_step(self):
+        for d, h in zip(self.dev_in, self.host_in):
+            d.copy_(h, non_blocking=True)
+        x, lens, pos, ids = self.dev_in
+        yy = self.model.decode_step(x, self.cache, lens, pos, ids)
+        self.y_host.copy_(yy, non_blocking=True)
+
+
+class PrefillRunner:
+    def __init__(self, inp, dev):
+        import numpy as np
+        import torch
+        sys.path.insert(0, os.path.join(ROOT, "tests"))
+        from gpu_pipeline import make_model
+        from gated_mla_b200 import LatentCache
+        w = self.w = inp["workload"]
+        self.dev = dev
+        dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+        self.model = make_model(inp, device=dev)
+        lens = [int(L) for L in inp["lengths"]]
+        self.max_len = max(lens)
+        self.cache = LatentCache(data=torch.zeros(len(lens), self.max_len, w.row, dtype=dt, device=dev))
+        self.x = torch.from_numpy(inp["x"]).to(dev, dt)
+        self.cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32, device=dev)
+        self.positions = torch.from_numpy(np.concatenate([np.arange(L) for L in lens]).astype(np.int32)).to(dev)
+        self.seq_ids = torch.from_numpy(
+            np.concatenate([np.full(L, b) for b, L in enumerate(lens)]).astype(np.int32)).to(dev)
+        T = self.x.shape[0]
+        self.q = torch.empty(T, w.n_heads, w.d_h + w.d_rope, dtype=dt, device=dev)
+        self.g = torch.empty(T, w.gate_width, dtype=torch.float32, device=dev)
+        self.o = torch.empty(T, w.n_heads * w.d_h, dtype=dt, device=dev)
+        self.y = torch.empty(T, w.d_model, dtype=dt, device=dev)
+        self.kernel_work = prefill_flops(w, lens)
+        self.work = sum(self.kernel_work.values())
+        self.dominant = None   # picked from the measured kernel times
+        self.host_in = [t.cpu().pin_memory() for t in (self.x, self.positions, self.seq_ids, self.cu)]
+        self.dev_in = [torch.empty_like(t) for t in (self.x, self.positions, self.seq_ids, self.cu)]
+        self.y_host = torch.empty(T, w.d_model, dtype=dt).pin_memory()
+
+    def step(self):
+        m = self.model
+        m.latent_project(self.x, self.positions, self.seq_ids, self.cache, q_out=self.q, gate_logits=self.g)
+        m.prefill(self.q, self.g, self.cache, self.cu, self.max_len, o_out=self.o)
+        m.gate_out(self.o, y_out=self.y)
+
+    def e2e_step(self):
+        for d, h in zip(self.dev_in, self.host_in):
+            d.copy_(h, non_blocking=True)
+        x, pos, ids, cu = self.dev_in
+        yy = self.model.prefill_step(x, self.cache, cu, self.max_len, pos, ids)
+        self.y_host.copy_(yy, non_blocking=True)
+
+
 def run_ours(args):
-    import numpy as np
     import torch
     import torch.distributed as dist
 
     import synth
     from gated_mla_b200 import _lib
-    sys.path.insert(0, os.path.join(ROOT, "tests"))
-    from gpu_pipeline import make_decode_cache, make_model
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -240,34 +368,18 @@ def run_ours(args):
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=180), device_id=dev)
 
-    w = synth.workload(WORKLOAD)
+    w = synth.workload(args.workload)
     inp = synth.generate(w, seed=0)
-    lens_np = inp["lengths"]
-    latent_bytes = int(lens_np.sum()) * w.row * 2
-    model = make_model(inp, device=dev)
-    cache = make_decode_cache(inp, device=dev, paged=False, fill=0.0)
-    B = w.batch
-    x = torch.from_numpy(inp["x"]).to(dev, torch.bfloat16)
-    seq_lens = torch.tensor(lens_np, dtype=torch.int32, device=dev)
-    positions = (seq_lens - 1).contiguous()
-    seq_ids = torch.arange(B, dtype=torch.int32, device=dev)
-    q = torch.empty(B, w.n_heads, w.d_h + w.d_rope, dtype=torch.bfloat16, device=dev)
-    g = torch.empty(B, w.gate_width, dtype=torch.float32, device=dev)
-    o = torch.empty(B, w.n_heads * w.d_h, dtype=torch.bfloat16, device=dev)
-    y = torch.empty(B, w.d_model, dtype=torch.bfloat16, device=dev)
+    run = DecodeRunner(inp, dev) if w.mode == "decode" else PrefillRunner(inp, dev)
+    scale, unit = work_unit(w)
     flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=dev)
 
-    def step():
-        model.latent_project(x, positions, seq_ids, cache, q_out=q, gate_logits=g)
-        model.decode(q, g, cache, seq_lens, o_out=o)
-        model.gate_out(o, y_out=y)
-
     # eager warm-up (also sizes the workspaces) and launches per step
-    step()
+    run.step()
     torch.cuda.synchronize()
-    model.sync_status()
+    run.model.sync_status()
     n0 = _lib.gmla_launch_count()
-    step()
+    run.step()
     torch.cuda.synchronize()
     launches_per_step = _lib.gmla_launch_count() - n0
 
@@ -275,11 +387,11 @@ def run_ours(args):
     s = torch.cuda.Stream(device=dev)
     s.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(s):
-        step()
+        run.step()
     torch.cuda.current_stream().wait_stream(s)
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
-        step()
+        run.step()
     torch.cuda.synchronize()
 
     stream = torch.cuda.current_stream()
@@ -287,7 +399,7 @@ def run_ours(args):
         flush.zero_()
         graph.replay()
     torch.cuda.synchronize()
-    model.sync_status()
+    run.model.sync_status()
 
     K = args.steps
     ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
@@ -312,23 +424,21 @@ def run_ours(args):
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    times = [a.elapsed_time(b) for a, b in zip(ev0, ev1)]
-    total_ms = sum(times)
+    total_ms = sum(a.elapsed_time(b) for a, b in zip(ev0, ev1))
     tt = torch.tensor([total_ms], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
     max_total_ms = float(tt.item())
-    value = world * latent_bytes * K / (max_total_ms / 1e3) / 1e9
-    model.sync_status()
+    value = world * run.work * K / (max_total_ms / 1e3) / scale
+    run.model.sync_status()
 
-    # dominant kernel: per-launch CUDA events on the launching stream. The step is
-    # captured with the library's event records inside the graph, so the records
-    # bracket the kernel nodes with no host time in between; each replay
-    # overwrites them and they are read after it.
+    # per-kernel times: the step captured with the library's event records inside
+    # the graph (no host time between a record and its kernel); each replay
+    # overwrites the records and they are read after it
     _lib.gmla_profile_enable(1)
     pgraph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(pgraph):
-        step()
+        run.step()
     torch.cuda.synchronize()
     n_rec = _lib.gmla_profile_count()
     by = {}
@@ -341,67 +451,64 @@ def run_ours(args):
             by.setdefault(name, []).append(ms)
     _lib.gmla_profile_enable(0)
     del pgraph
-    attn_ms = statistics.mean(by["decode_attn"])
-    achieved = latent_bytes / (attn_ms / 1e3) / 1e9
-    pk = peaks()
     kernel_ms = {k: statistics.mean(v) * (len(v) // K) for k, v in by.items()}   # per step
+    pk = peaks()
+    if w.mode == "decode":
+        dom = "decode_attn"
+        achieved = run.kernel_work[dom] / (kernel_ms[dom] / 1e3) / 1e9
+        roof = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / pk["hbm_gbs"], "peak_source": pk["source"],
+                "traffic": ncu_traffic() if args.workload == DEFAULT_WORKLOAD else None,
+                "launch_ms": kernel_ms[dom], "algorithmic_bytes_per_launch": run.kernel_work[dom]}
+    else:
+        per = {k: v for k, v in run.kernel_work.items() if k in kernel_ms}
+        if not per:   # fp32 path: its kernels are not split the same way; use the whole step
+            per = {"step": run.work}
+            kernel_ms["step"] = max_total_ms / K
+        dom = max(per, key=lambda k: kernel_ms[k])
+        achieved = per[dom] / (kernel_ms[dom] / 1e3) / 1e12
+        roof = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": pk["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"], "peak_source": pk["source"] + " burst",
+                "traffic": None, "launch_ms": kernel_ms[dom], "algorithmic_flops_per_launch": per[dom],
+                "per_kernel_tflops": {k: per[k] / (kernel_ms[k] / 1e3) / 1e12 for k in per}}
 
     # end to end through the public API, host buffers (pinned), copies inside the events
-    x_h = torch.from_numpy(inp["x"]).to(torch.bfloat16).pin_memory()
-    lens_h = torch.tensor(lens_np, dtype=torch.int32).pin_memory()
-    pos_h = (lens_h - 1).pin_memory()
-    ids_h = torch.arange(B, dtype=torch.int32).pin_memory()
-    y_h = torch.empty(B, w.d_model, dtype=torch.bfloat16).pin_memory()
-    x_d, lens_d, pos_d, ids_d = (torch.empty_like(t, device=dev) for t in (x_h, lens_h, pos_h, ids_h))
-    h2d = sum(t.numel() * t.element_size() for t in (x_h, lens_h, pos_h, ids_h))
-    d2h = y_h.numel() * y_h.element_size()
-
-    def e2e_step():
-        x_d.copy_(x_h, non_blocking=True)
-        lens_d.copy_(lens_h, non_blocking=True)
-        pos_d.copy_(pos_h, non_blocking=True)
-        ids_d.copy_(ids_h, non_blocking=True)
-        yy = model.decode_step(x_d, cache, lens_d, pos_d, ids_d)
-        y_h.copy_(yy, non_blocking=True)
-
+    h2d = sum(t.numel() * t.element_size() for t in run.host_in)
+    d2h = run.y_host.numel() * run.y_host.element_size()
     for _ in range(3):
-        e2e_step()
+        run.e2e_step()
     torch.cuda.synchronize()
     e0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     e1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     for i in range(K):
         flush.zero_()
         e0[i].record(stream)
-        e2e_step()
+        run.e2e_step()
         e1[i].record(stream)
     torch.cuda.synchronize()
     e2e_ms = sum(a.elapsed_time(b) for a, b in zip(e0, e1))
     et = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(et, op=dist.ReduceOp.MAX)
-    e2e_value = world * latent_bytes * K / (float(et.item()) / 1e3) / 1e9
-    model.sync_status()
+    e2e_value = world * run.work * K / (float(et.item()) / 1e3) / scale
+    run.model.sync_status()
 
     cpu = None
     if rank == 0 and not args.no_cpu_baseline:
-        nb, sec, seqs = oracle_sample(inp, args.cpu_seconds)
-        cpu = {"value": nb / sec / 1e9, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-               "sample": f"{len(seqs)} of {B} sequences ({nb / 1e6:.1f} MB of latent rows) of the same workload, "
-                         f"fp64 explicit form, numpy/BLAS, {sec:.1f} s"}
+        wk, sec, desc = oracle_sample(inp, args.cpu_seconds)
+        cpu = {"value": wk / sec / scale, "unit": unit, "cores": blas_threads(), "kind": "oracle",
+               "sample": f"{desc} of the same workload, fp64 explicit form, numpy/BLAS, {sec:.1f} s"}
     if world > 1:
         dist.barrier()
     if rank == 0:
         line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
-            "ms_per_step": max_total_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16", "data": "synthetic", "config": dict(config_dict(w, inp), cuda_graph=True),
-            "roofline": {"bound": "hbm", "kernel": "decode_attn", "achieved": achieved, "peak": pk["hbm_gbs"],
-                         "unit": "GB/s", "frac": achieved / pk["hbm_gbs"], "peak_source": pk["source"],
-                         "traffic": ncu_traffic(), "launch_ms": attn_ms,
-                         "algorithmic_bytes_per_launch": latent_bytes},
-            "kernel_ms": kernel_ms,
-            "cpu_baseline": cpu,
-            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "metric": DECODE_METRIC if w.mode == "decode" else PREFILL_METRIC, "value": value, "unit": unit,
+            "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": max_total_ms / K,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
+            "config": dict(config_dict(w, inp), cuda_graph=True),
+            "roofline": roof, "kernel_ms": kernel_ms, "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": int(launches_per_step * K),
             "clocks": clk.summary(),
         }

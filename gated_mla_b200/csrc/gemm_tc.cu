@@ -384,12 +384,12 @@ __global__ void __launch_bounds__(192, 1) gemm_bf16_tc_kernel(const __grid_const
 }
 
 template <int BN, bool kSwap>
-static cudaError_t launch_one(const GemmArgs& a, dim3 grid, cudaStream_t st) {
+static cudaError_t launch_one(const GemmArgs& a, dim3 grid, cudaStream_t st, const char* name) {
   using C = GemmCfg<BN>;
   auto k = gemm_bf16_tc_kernel<BN, kSwap>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
-  prof_begin(st, kSwap ? "gemm_bf16_swap" : "gemm_bf16");
+  prof_begin(st, name);
   if (kSwap && a.splits > 1) {
     // the K splits of one tile run as a cluster along z
     cudaLaunchConfig_t cfg{};
@@ -439,21 +439,22 @@ SwapPlan gemm_swap_plan(int wtiles, int T, int K, int num_sms) {
   return p;
 }
 
-cudaError_t launch_gemm_bf16(const GemmArgs& a, bool swap, int bn, int token_tiles, cudaStream_t st) {
+cudaError_t launch_gemm_bf16(const GemmArgs& a, bool swap, int bn, int token_tiles, cudaStream_t st,
+                             const char* name) {
   dim3 grid(a.seg_tile_begin[a.n_seg], token_tiles, swap ? (a.splits > 1 ? a.splits : 1) : 1);
   if (grid.x == 0 || grid.y == 0) return cudaSuccess;
   if (swap) {
     switch (bn) {
-      case 16: return launch_one<16, true>(a, grid, st);
-      case 32: return launch_one<32, true>(a, grid, st);
-      case 64: return launch_one<64, true>(a, grid, st);
-      case 128: return launch_one<128, true>(a, grid, st);
-      case 256: return launch_one<256, true>(a, grid, st);
+      case 16: return launch_one<16, true>(a, grid, st, name);
+      case 32: return launch_one<32, true>(a, grid, st, name);
+      case 64: return launch_one<64, true>(a, grid, st, name);
+      case 128: return launch_one<128, true>(a, grid, st, name);
+      case 256: return launch_one<256, true>(a, grid, st, name);
     }
   } else {
     switch (bn) {
-      case 128: return launch_one<128, false>(a, grid, st);
-      case 256: return launch_one<256, false>(a, grid, st);
+      case 128: return launch_one<128, false>(a, grid, st, name);
+      case 256: return launch_one<256, false>(a, grid, st, name);
     }
   }
   return cudaErrorInvalidValue;

@@ -427,7 +427,7 @@ gmla_status gmla_latent_project(const gmla_config* cfg, const gmla_weights* w, c
   const int ttiles = swap ? sp.ttiles : (T + 127) / 128;
   cudaError_t e = cudaSuccess;
   if (swap) e = set_splits(a, sp, static_cast<uint8_t*>(workspace) + 256, st);
-  if (e == cudaSuccess) e = launch_gemm_bf16(a, swap, bn, ttiles, st);
+  if (e == cudaSuccess) e = launch_gemm_bf16(a, swap, bn, ttiles, st, "gemm_project");
   return e == cudaSuccess ? GMLA_OK : cuda_fail(e, "latent_project");
 }
 
@@ -556,7 +556,7 @@ gmla_status gmla_decode(const gmla_config* cfg, const gmla_weights* w, const voi
   g.status = status;
 
   cudaError_t e = launch_decode_bf16(a, st);
-  if (e == cudaSuccess) e = launch_gemm_bf16(g, true, sp.bn, sp.ttiles, st);
+  if (e == cudaSuccess) e = launch_gemm_bf16(g, true, sp.bn, sp.ttiles, st, "gemm_wv_gate");
   return e == cudaSuccess ? GMLA_OK : cuda_fail(e, "decode");
 }
 
@@ -646,7 +646,7 @@ gmla_status gmla_prefill(const gmla_config* cfg, const gmla_weights* w, const vo
   g.act_seq_stride = cache->capacity;
   g.cu_seqlens = cu_seqlens;
   g.status = status;
-  cudaError_t e = launch_gemm_bf16(g, false, bn, B * tps, st);
+  cudaError_t e = launch_gemm_bf16(g, false, bn, B * tps, st, "gemm_kv");
   if (e != cudaSuccess) return cuda_fail(e, "prefill K/V rebuild");
 
   PrefillArgs p{};
@@ -732,7 +732,7 @@ gmla_status gmla_gate_out(const gmla_config* cfg, const gmla_weights* w, const v
   const int ttiles = swap ? sp.ttiles : (T + 127) / 128;
   cudaError_t e = cudaSuccess;
   if (swap) e = set_splits(a, sp, static_cast<uint8_t*>(workspace) + 256 + align256(static_cast<size_t>(T) * HD * 2), st);
-  if (e == cudaSuccess) e = launch_gemm_bf16(a, swap, bn, ttiles, st);
+  if (e == cudaSuccess) e = launch_gemm_bf16(a, swap, bn, ttiles, st, "gemm_out");
   return e == cudaSuccess ? GMLA_OK : cuda_fail(e, "gate_out");
 }
 

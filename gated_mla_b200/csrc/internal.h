@@ -10,7 +10,8 @@
 namespace gmla {
 
 // ----- tcgen05 GEMM (gemm_tc.cu) -----
-cudaError_t launch_gemm_bf16(const GemmArgs& a, bool swap, int bn, int token_tiles, cudaStream_t st);
+cudaError_t launch_gemm_bf16(const GemmArgs& a, bool swap, int bn, int token_tiles, cudaStream_t st,
+                             const char* name);
 int gemm_weight_tile(bool swap, int bn);
 int gemm_swap_bn(int T);
 // Tiling of the swap orientation (few tokens): token tile width, K splits and

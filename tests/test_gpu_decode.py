@@ -130,3 +130,26 @@ def test_decode_full_paged_config_sampled():
     gpu = run_decode(inp)
     seqs = sorted(np.random.default_rng(0).choice(64, 8, replace=False).tolist())
     _check(inp, gpu, seqs=seqs)
+
+
+@pytest.mark.slow
+def test_decode_full_long_context_rope_sampled():
+    """The long-context workload (batch 8 x 131072 cached rows, H 128, d_c 512 +
+    decoupled RoPE 64). The oracle evaluates y of one sequence in the absorbed
+    form (pinned equal to the explicit form by the oracle's own tests) and the
+    explicit per-head output o of two (sequence, head) pairs."""
+    inp = synth.generate(synth.workload("decode_long_rope"), seed=0)
+    gpu = run_decode(inp)
+    w = inp["workload"]
+    p = oracle.params(inp)
+    # y of sequence 3, all heads (absorbed form)
+    ref = oracle.decode(p, inp["x"], inp["past"], seqs=[3], absorbed=True)
+    assert_close(gpu["q"][:, :, :w.d_h], ref["q"], BF16_TOL, "q")
+    assert_close(gpu["q"][:, :, w.d_h:], ref["qR"], BF16_TOL, "qR (rotated at position 131071)")
+    assert_close(gpu["o"][[3]], ref["gated"], BF16_TOL, "gated o, sequence 3")
+    assert_close(gpu["y"][[3]], ref["y"], BF16_TOL, "y, sequence 3")
+    # explicit form for two single heads
+    for b, h in ((0, 5), (7, 127)):
+        ex = oracle.decode(p, inp["x"], inp["past"], seqs=[b], heads=[h])
+        g = oracle.sigmoid(ex["glogit"][b, h * w.d_h:(h + 1) * w.d_h])
+        assert_close(gpu["o"][b, h * w.d_h:(h + 1) * w.d_h], g * ex["o"][0, 0], BF16_TOL, f"o[{b}, head {h}]")
