@@ -15,8 +15,8 @@ over whole prompts; its metric is explicit-form algorithmic FLOPs per second
 (TFLOP/s). Inputs are synthetic, drawn by ``synth``.
 
 Timing: W untimed warm-up steps; then K steps, each replayed from a CUDA
-graph between CUDA events on the launching stream, with a 256 MiB memset
-flushing L2 before every step (outside the events); barrier + synchronize on
+graph between CUDA events on the launching stream, with L2 flushed before
+every step by a 256 MiB memset and a read of it (outside the events); barrier + synchronize on
 both sides; the max over ranks of the summed step times. Under torchrun every
 rank runs its own replica of the workload (weak scaling; no data-path
 collective). Rank 0 prints one JSON line.
@@ -45,6 +45,14 @@ PREFILL_METRIC = "Gated-MLA prefill TFLOP/s (latent_project + prefill + gate_out
 DEFAULT_WORKLOAD = "decode_b32"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 
+
+
+def flush_l2(buf):
+    """Evicts L2 between timed steps: a write of a buffer twice the size of L2,
+    then a read of it, so the next step finds none of its inputs cached and no
+    dirty line left to write back on its time."""
+    buf.zero_()
+    buf.sum()
 
 def parse():
     ap = argparse.ArgumentParser()
@@ -180,7 +188,7 @@ def config_dict(w, inp):
         extra = {"flops_per_step": sum(prefill_flops(w, lens).values())}
     return dict({"workload": desc, "batch": w.batch, "d_model": w.d_model, "n_heads": w.n_heads, "d_h": w.d_h,
                  "d_c": w.d_c, "d_rope": w.d_rope,
-                 "l2": "flushed before every timed step (256 MiB memset, outside the events)",
+                 "l2": "flushed before every timed step (256 MiB memset then a read of it, outside the events)",
                  "parallelism": "replica per GPU"}, **extra)
 
 
@@ -396,7 +404,7 @@ def run_ours(args):
 
     stream = torch.cuda.current_stream()
     for _ in range(max(3, args.warmup)):
-        flush.zero_()
+        flush_l2(flush)
         graph.replay()
     torch.cuda.synchronize()
     run.model.sync_status()
@@ -410,7 +418,7 @@ def run_ours(args):
     with ClockSampler(local) as clk:
         t_wall = time.perf_counter()
         for i in range(K):
-            flush.zero_()
+            flush_l2(flush)
             ev0[i].record(stream)
             graph.replay()
             ev1[i].record(stream)
@@ -418,7 +426,7 @@ def run_ours(args):
         # keep the GPU busy long enough for the clock sampler to see it
         extra = 0
         while time.perf_counter() - t_wall < 1.0 and extra < 20000:
-            flush.zero_()
+            flush_l2(flush)
             graph.replay()
             extra += 1
         torch.cuda.synchronize()
@@ -443,7 +451,7 @@ def run_ours(args):
     n_rec = _lib.gmla_profile_count()
     by = {}
     for _ in range(K):
-        flush.zero_()
+        flush_l2(flush)
         pgraph.replay()
         torch.cuda.synchronize()
         for i in range(n_rec):
@@ -481,7 +489,7 @@ def run_ours(args):
     e0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     e1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     for i in range(K):
-        flush.zero_()
+        flush_l2(flush)
         e0[i].record(stream)
         run.e2e_step()
         e1[i].record(stream)

@@ -284,66 +284,75 @@ __global__ void __launch_bounds__(192, 1) decode_attn_kernel(const __grid_consta
 
   if (warp == 0) {
     // ------------------------------ TMA producer ------------------------------
+    // The whole warp walks the loop: lane 0 waits for free slots and arms the
+    // barriers; with a paged cache lane r reads the page of chunk r of the
+    // tile (one coalesced read per tile) and issues that chunk's copy.
     if (lane == 0) {
       tma_prefetch_desc(&a.cache_map);
       tma_prefetch_desc(&a.qa_map);
-      const uint64_t pol_c = a.n_hg > 1 ? l2_evict_normal() : l2_evict_first();
-      const uint64_t pol_q = l2_evict_last();
-      uint32_t nbox = 0, nrope = 0, nq = 0;
-      bool ok = true;
-      for (int si = seg_lo; si < seg_hi && ok; ++si) {
-        const int4 sg = a.seg_info[si];
-        const int b = sg.x;
-        const int L = a.seq_lens[b];
-        if (nq > 0 && !mbar_wait(&sm->q_empty, (nq - 1) & 1, abort_flag, a.status)) { ok = false; break; }
-        mbar_arrive_expect_tx(&sm->q_full, C::kQBytes);
-        for (int j = 0; j < NBOX; ++j)
-          tma_load_2d(&a.qa_map, &sm->q_full, qs + j * HG * 128, j * 64, b * a.H + hg * HG, pol_q);
-        ++nq;
-        for (int t = sg.y; t < sg.z && ok; ++t) {
-          const int tok0 = t * kTileTok;
-          const int valid = min(kTileTok, L - tok0);
-          for (int j = 0; j < NBOX; ++j) {
-            uint64_t* bar;
-            uint8_t* dst;
-            if (j < kNcBox) {
-              const uint32_t slot = nbox % NR;
+    }
+    const uint64_t pol_c = a.n_hg > 1 ? l2_evict_normal() : l2_evict_first();
+    const uint64_t pol_q = l2_evict_last();
+    const bool paged = a.cache.paged != 0;
+    const int ps = paged ? a.cache.page_size : kTileTok;
+    uint32_t nbox = 0, nrope = 0, nq = 0;
+    bool ok = true;
+    for (int si = seg_lo; si < seg_hi && ok; ++si) {
+      const int4 sg = a.seg_info[si];
+      const int b = sg.x;
+      const int L = a.seq_lens[b];
+      if (lane == 0) {
+        if (nq > 0 && !mbar_wait(&sm->q_empty, (nq - 1) & 1, abort_flag, a.status)) ok = false;
+        if (ok) {
+          mbar_arrive_expect_tx(&sm->q_full, C::kQBytes);
+          for (int j = 0; j < NBOX; ++j)
+            tma_load_2d(&a.qa_map, &sm->q_full, qs + j * HG * 128, j * 64, b * a.H + hg * HG, pol_q);
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      ++nq;
+      for (int t = sg.y; t < sg.z && ok; ++t) {
+        const int tok0 = t * kTileTok;
+        const int valid = min(kTileTok, L - tok0);
+        const int nchunk = ps >= kTileTok ? 1 : (valid + ps - 1) / ps;   // <= 16 (page size >= 8)
+        int page = 0;
+        if (paged && lane < nchunk)
+          page = a.cache.block_table[static_cast<int64_t>(b) * a.cache.max_pages_per_seq + (tok0 + lane * ps) / ps];
+        const uint32_t tx = ps >= kTileTok ? kBoxBytes : nchunk * ps * 128;
+        for (int j = 0; j < NBOX; ++j) {
+          const bool ring_box = j < kNcBox;
+          const uint32_t slot = nbox % NR;
+          uint64_t* bar = ring_box ? &sm->full[slot] : &sm->rope_full;
+          uint8_t* dst = ring_box ? ring + slot * kBoxBytes : rope_slot;
+          if (lane == 0) {
+            if (ring_box) {
               if (nbox >= static_cast<uint32_t>(NR) &&
-                  !mbar_wait(&sm->empty[slot], ((nbox / NR) & 1) ^ 1, abort_flag, a.status)) { ok = false; break; }
-              bar = &sm->full[slot];
-              dst = ring + slot * kBoxBytes;
-              ++nbox;
-            } else {
-              if (nrope > 0 && !mbar_wait(&sm->rope_empty, (nrope - 1) & 1, abort_flag, a.status)) { ok = false; break; }
-              bar = &sm->rope_full;
-              dst = rope_slot;
-              ++nrope;
+                  !mbar_wait(&sm->empty[slot], ((nbox / NR) & 1) ^ 1, abort_flag, a.status))
+                ok = false;
+            } else if (nrope > 0 && !mbar_wait(&sm->rope_empty, (nrope - 1) & 1, abort_flag, a.status)) {
+              ok = false;
             }
-            if (!a.cache.paged) {
-              mbar_arrive_expect_tx(bar, kBoxBytes);
-              tma_load_2d(&a.cache_map, bar, dst, j * 64, b * a.cache.capacity + tok0, pol_c);
-            } else {
-              const int ps = a.cache.page_size;
-              const int32_t* bt = a.cache.block_table + static_cast<int64_t>(b) * a.cache.max_pages_per_seq;
-              if (ps >= kTileTok) {
-                mbar_arrive_expect_tx(bar, kBoxBytes);
-                tma_load_3d(&a.cache_map, bar, dst, j * 64, tok0 % ps, bt[tok0 / ps], pol_c);
-              } else {
-                const int nchunk = (valid + ps - 1) / ps;
-                mbar_arrive_expect_tx(bar, nchunk * ps * 128);
-                for (int r = 0; r < nchunk; ++r)
-                  tma_load_3d(&a.cache_map, bar, dst + r * ps * 128, j * 64, 0, bt[(tok0 + r * ps) / ps], pol_c);
-              }
-            }
+            if (ok) mbar_arrive_expect_tx(bar, tx);
+          }
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          if (!ok) break;
+          if (ring_box) ++nbox; else ++nrope;
+          if (!paged) {
+            if (lane == 0) tma_load_2d(&a.cache_map, bar, dst, j * 64, b * a.cache.capacity + tok0, pol_c);
+          } else if (ps >= kTileTok) {
+            if (lane == 0) tma_load_3d(&a.cache_map, bar, dst, j * 64, tok0 % ps, page, pol_c);
+          } else if (lane < nchunk) {
+            tma_load_3d(&a.cache_map, bar, dst + lane * ps * 128, j * 64, 0, page, pol_c);
           }
         }
       }
-      if (*abort_flag) {   // let issued copies land before the block exits
-        for (uint32_t c = nbox > static_cast<uint32_t>(NR) ? nbox - NR : 0; c < nbox; ++c)
-          mbar_drain(&sm->full[c % NR], (c / NR) & 1);
-        if (nrope) mbar_drain(&sm->rope_full, (nrope - 1) & 1);
-        if (nq) mbar_drain(&sm->q_full, (nq - 1) & 1);
-      }
+    }
+    if (lane == 0 && *abort_flag) {   // let issued copies land before the block exits
+      for (uint32_t c = nbox > static_cast<uint32_t>(NR) ? nbox - NR : 0; c < nbox; ++c)
+        mbar_drain(&sm->full[c % NR], (c / NR) & 1);
+      if (nrope) mbar_drain(&sm->rope_full, (nrope - 1) & 1);
+      if (nq) mbar_drain(&sm->q_full, (nq - 1) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------ MMA issuer ------------------------------
