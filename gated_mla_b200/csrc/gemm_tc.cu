@@ -30,6 +30,9 @@ struct GemmCfg {
   static constexpr int kStages = (BN >= 256) ? 4 : (BN >= 128 ? 6 : 4);
   static constexpr int kTmemCols = BN < 32 ? 32 : BN;
   static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/ + 12 * BN;
+  // split-K partials are received into the (then idle) stage memory:
+  // splits x 128 x cpr fp32 with splits <= 8 and cpr = ceil4(ceil(BN / splits)) <= BN / splits + 3
+  static_assert(128 * 4 * (BN + 24) <= kStages * kStageBytes, "split-K receive buffer");
 };
 
 struct GemmTile {
@@ -78,7 +81,8 @@ __global__ void __launch_bounds__(192, 1) gemm_bf16_tc_kernel(const __grid_const
   uint64_t* empty = full + C::kStages;
   uint64_t* acc_full = empty + C::kStages;
   uint64_t* drain = acc_full + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* red_full = drain + 1;   // split-K: the partials addressed to this CTA have landed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(red_full + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   // per-token output row and position of this tile (swap orientation), filled once
   int64_t* tok_row = reinterpret_cast<int64_t*>(smem + C::kStages * C::kStageBytes + 256);
@@ -96,6 +100,12 @@ __global__ void __launch_bounds__(192, 1) gemm_bf16_tc_kernel(const __grid_const
   const int kbps = (kSwap && a.kb_per_split > 0) ? a.kb_per_split : num_kb_total;
   const int kb_begin = kSwap ? blockIdx.z * kbps : 0;
   const int num_kb = kSwap ? min(num_kb_total - kb_begin, kbps) : num_kb_total;
+  // split-K (swap orientation): the K splits of a tile form a cluster along z;
+  // rank z owns the accumulator columns [z*cpr, (z+1)*cpr) of the tile
+  const bool split = kSwap && a.splits > 1;
+  const int cpr = ((BN + a.splits - 1) / a.splits + 3) & ~3;
+  const uint32_t rank = split ? cluster_ctarank() : 0u;
+  const int own_cols = split ? max(0, min(cpr, BN - static_cast<int>(rank) * cpr)) : 0;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::kStages; ++i) {
@@ -104,8 +114,10 @@ __global__ void __launch_bounds__(192, 1) gemm_bf16_tc_kernel(const __grid_const
     }
     mbar_init(acc_full, 1);
     mbar_init(drain, 1);
+    mbar_init(red_full, 1);
     *abort_flag = 0;
     fence_mbar_init();
+    if (split) mbar_arrive_expect_tx(red_full, a.splits * 128 * own_cols * 4);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::kTmemCols);
@@ -232,7 +244,7 @@ __global__ void __launch_bounds__(192, 1) gemm_bf16_tc_kernel(const __grid_const
               static_cast<__nv_bfloat16*>(e.out)[off] = __float2bfloat16_rn(val);
           }
         };
-        if (a.splits <= 1) {
+        if (!split) {
 #pragma unroll 1
           for (int c0 = 0; c0 < BN; c0 += 16) {
             uint32_t v[16];
@@ -243,25 +255,8 @@ __global__ void __launch_bounds__(192, 1) gemm_bf16_tc_kernel(const __grid_const
             for (int j = 0; j < 16; ++j) x[j] = __uint_as_float(v[j]);
             if (acc_ok) store_chunk(c0, x);
           }
-        } else {
-          // K splits of this tile form one cluster: every split leaves its fp32
-          // partial in its own (now idle) stage memory, rank 0 sums them over
-          // distributed shared memory and stores. Both cluster barriers are
-          // reached on every path so no CTA waits for one that left.
-          float* part = reinterpret_cast<float*>(smem) + r * (BN + 4);   // [128][BN + 4]
-#pragma unroll 1
-          for (int c0 = 0; c0 < BN; c0 += 16) {
-            uint32_t v[16];
-            tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + c0, v);
-            tmem_ld_wait();
-#pragma unroll
-            for (int j = 0; j < 16; j += 4)
-              *reinterpret_cast<float4*>(part + c0 + j) =
-                  acc_ok ? make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]), __uint_as_float(v[j + 2]),
-                                       __uint_as_float(v[j + 3]))
-                         : make_float4(0.f, 0.f, 0.f, 0.f);
-          }
         }
+        // (split-K: the accumulator is pushed to the owning CTAs below)
       } else {
         // row r = token, columns = weight features
         const bool tok_ok = r < tile.ntok;
@@ -320,59 +315,81 @@ __global__ void __launch_bounds__(192, 1) gemm_bf16_tc_kernel(const __grid_const
     }
   }
 
-  if (kSwap && a.splits > 1) {
-    cluster_sync_all();   // every split's partial is in its shared memory
-    // reduce-scatter: rank z sums columns [z*cpr, (z+1)*cpr) of every split's
-    // partial (one float4 per split per row, all loads in flight together)
-    // and stores them
-    const int cpr = ((BN + a.splits - 1) / a.splits + 3) & ~3;
-    const int col0 = static_cast<int>(cluster_ctarank()) * cpr;
-    if (warp >= 2 && col0 < BN) {
+  if (split) {
+    // Every split of the tile has finished its MMAs once the cluster barrier
+    // completes, so their stage memory is idle and receives the partials:
+    // recv[src split][row][cpr] fp32. Each split pushes the columns that rank
+    // z owns straight from its accumulator to rank z (st.async, completing
+    // bytes on rank z's red_full); the owner sums the splits and stores. A CTA
+    // leaves only after everything addressed to it has landed, and what it
+    // sends comes from registers, so no second cluster barrier is needed.
+    cluster_sync_all();
+    float* recv = reinterpret_cast<float*>(smem);
+    if (warp >= 2) {
       const int q = warp & 3, r = q * 32 + lane;
-      const int f = tile.wrow0 + r;
-      const EpiSeg e = a.epi[tile.seg];
-      const int seg_rows = a.seg_rows[tile.seg];
-      const bool f_ok = f < seg_rows;
-      const int64_t colpart = static_cast<int64_t>(f / e.block) * e.block_stride + (f % e.block) + e.col_offset;
-      const float fbias = (e.bias && f_ok) ? e.bias[f] : 0.f;
-      const int gcol = e.gate ? f / e.gate_div : 0;
-      const uint32_t part = smem_u32(smem) + r * (BN + 4) * 4;
+      const bool acc_ok = !*abort_flag;
+      tc_fence_after();
 #pragma unroll 1
-      for (int c0 = col0; c0 < min(BN, col0 + cpr); c0 += 4) {
-        float4 u[8];
+      for (int c0 = 0; c0 < BN; c0 += 16) {
+        uint32_t v[16];
+        tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + c0, v);
+        tmem_ld_wait();
 #pragma unroll
-        for (int z = 0; z < 8; ++z)
-          u[z] = z < a.splits ? ld_cluster_f4(cluster_map(part, z) + c0 * 4) : make_float4(0.f, 0.f, 0.f, 0.f);
-        float x[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int z = 0; z < 8; ++z) {
-          x[0] += u[z].x;
-          x[1] += u[z].y;
-          x[2] += u[z].z;
-          x[3] += u[z].w;
+        for (int g = 0; g < 16; g += 4) {
+          const int col = c0 + g;
+          const uint32_t z = static_cast<uint32_t>(col / cpr);
+          const float4 x = acc_ok ? make_float4(__uint_as_float(v[g]), __uint_as_float(v[g + 1]),
+                                                __uint_as_float(v[g + 2]), __uint_as_float(v[g + 3]))
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+          const uint32_t dst = smem_u32(recv + (rank * 128 + r) * cpr + (col - static_cast<int>(z) * cpr));
+          st_async_v4(cluster_map(dst, z), x, cluster_map(smem_u32(red_full), z));
         }
+      }
+      if (own_cols > 0) {
+        const bool got = mbar_wait_cluster(red_full, 0, abort_flag, a.status);
+        const int col0 = static_cast<int>(rank) * cpr;
+        const int f = tile.wrow0 + r;
+        const EpiSeg e = a.epi[tile.seg];
+        const int seg_rows = a.seg_rows[tile.seg];
+        const bool f_ok = f < seg_rows;
+        const int64_t colpart = static_cast<int64_t>(f / e.block) * e.block_stride + (f % e.block) + e.col_offset;
+        const float fbias = (e.bias && f_ok) ? e.bias[f] : 0.f;
+        const int gcol = e.gate ? f / e.gate_div : 0;
+#pragma unroll 1
+        for (int c = 0; c < own_cols; c += 4) {
+          float x[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int tl = c0 + j;
-          float val = x[j];
-          if (e.rope) {
-            const float partner = __shfl_xor_sync(0xffffffffu, val, 1);
-            const int fi = f % e.block;
-            val = rope_rotate(val, partner, fi & 1, tok_pos[tl], fi >> 1, e.block, a.log2_rope_base);
+          for (int z = 0; z < 8; ++z) {
+            if (z >= a.splits) break;
+            const float4 u = *reinterpret_cast<const float4*>(recv + (z * 128 + r) * cpr + c);
+            x[0] += u.x;
+            x[1] += u.y;
+            x[2] += u.z;
+            x[3] += u.w;
           }
-          const int64_t row = tok_row[tl];
-          if (row < 0 || !f_ok || *abort_flag) continue;
-          val += fbias;
-          if (e.gate) val *= 1.f / (1.f + __expf(-e.gate[static_cast<int64_t>(tile.tok0 + tl) * e.gate_stride + gcol]));
-          const int64_t off = row * e.row_stride + colpart;
-          if (e.out_f32)
-            static_cast<float*>(e.out)[off] = val;
-          else
-            static_cast<__nv_bfloat16*>(e.out)[off] = __float2bfloat16_rn(val);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int tl = col0 + c + j;
+            float val = x[j];
+            if (e.rope) {
+              const float partner = __shfl_xor_sync(0xffffffffu, val, 1);
+              const int fi = f % e.block;
+              val = rope_rotate(val, partner, fi & 1, tok_pos[tl], fi >> 1, e.block, a.log2_rope_base);
+            }
+            const int64_t row = tok_row[tl];
+            if (row < 0 || !f_ok || !got) continue;
+            val += fbias;
+            if (e.gate)
+              val *= 1.f / (1.f + __expf(-e.gate[static_cast<int64_t>(tile.tok0 + tl) * e.gate_stride + gcol]));
+            const int64_t off = row * e.row_stride + colpart;
+            if (e.out_f32)
+              static_cast<float*>(e.out)[off] = val;
+            else
+              static_cast<__nv_bfloat16*>(e.out)[off] = __float2bfloat16_rn(val);
+          }
         }
       }
     }
-    cluster_sync_all();   // rank 0 has finished reading the other splits' memory
   }
 
   tc_fence_before();
