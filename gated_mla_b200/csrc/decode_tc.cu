@@ -127,11 +127,13 @@ constexpr int kAbsorbB = 8;
 constexpr int kAbsorbCols = 64;
 constexpr int kAbsorbKG = 16;
 
-__global__ void __launch_bounds__(256) decode_absorb_plan_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(256, 4) decode_absorb_plan_kernel(DecodeArgs a) {
+  if (threadIdx.x == 0) griddep_launch_dependents();
   const int n_cblk = a.d_c / kAbsorbCols;
   const int n_bblk = (a.B + kAbsorbB - 1) / kAbsorbB;
   const int blk = blockIdx.x;
   if (blk == a.H * n_bblk * n_cblk) {
+    griddep_wait();
     decode_plan_block(a);
     return;
   }
@@ -144,38 +146,48 @@ __global__ void __launch_bounds__(256) decode_absorb_plan_kernel(DecodeArgs a) {
   const int row = a.d_c + a.d_rope;
   __shared__ float sq[kAbsorbB][256];
   __shared__ float red[kAbsorbKG][kAbsorbB][kAbsorbCols];
+  const int kg = threadIdx.x >> 4;             // 16 groups over d_h
+  const int cl = (threadIdx.x & 15) * 4;       // 4 columns of the block's 64
+  const int c0 = cb * kAbsorbCols + cl;
+  const int kper = (a.d_h + kAbsorbKG - 1) / kAbsorbKG;
+  const __nv_bfloat16* Wk = static_cast<const __nv_bfloat16*>(a.W_k) + static_cast<int64_t>(h) * a.d_h * a.d_c;
+  const int k_lo = kg * kper, k_hi = min(a.d_h, k_lo + kper);
+  // W_k is a weight (no kernel writes it): the first rows of this thread's
+  // slice are in flight before waiting for the kernel that produces the queries
+  constexpr int kChunk = 8;   // rows of W_k held in registers at a time
+  uint2 wv[kChunk];
+  auto load_w = [&](int k0) {
+#pragma unroll
+    for (int i = 0; i < kChunk; ++i)
+      if (k0 + i < k_hi) wv[i] = *reinterpret_cast<const uint2*>(Wk + static_cast<int64_t>(k0 + i) * a.d_c + c0);
+  };
+  load_w(k_lo);
+  griddep_wait();
   const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(a.q);
   for (int i = threadIdx.x; i < kAbsorbB * a.d_h; i += blockDim.x) {
     const int bi = i / a.d_h, k = i % a.d_h;
     sq[bi][k] = bi < nb ? __bfloat162float(q[(static_cast<int64_t>(b0 + bi) * a.H + h) * dq + k]) : 0.f;
   }
   __syncthreads();
-  const int kg = threadIdx.x >> 4;             // 16 groups over d_h
-  const int cl = (threadIdx.x & 15) * 4;       // 4 columns of the block's 64
-  const int c0 = cb * kAbsorbCols + cl;
-  const int kper = (a.d_h + kAbsorbKG - 1) / kAbsorbKG;
-  const __nv_bfloat16* Wk = static_cast<const __nv_bfloat16*>(a.W_k) + static_cast<int64_t>(h) * a.d_h * a.d_c;
   float acc[kAbsorbB][4];
 #pragma unroll
   for (int bi = 0; bi < kAbsorbB; ++bi)
 #pragma unroll
     for (int j = 0; j < 4; ++j) acc[bi][j] = 0.f;
-  const int k_lo = kg * kper, k_hi = min(a.d_h, k_lo + kper);
-  uint2 wv[16];
+  for (int k0 = k_lo; k0 < k_hi; k0 += kChunk) {
+    if (k0 != k_lo) load_w(k0);
 #pragma unroll
-  for (int i = 0; i < 16; ++i)
-    if (k_lo + i < k_hi) wv[i] = *reinterpret_cast<const uint2*>(Wk + static_cast<int64_t>(k_lo + i) * a.d_c + c0);
+    for (int i = 0; i < kChunk; ++i) {
+      if (k0 + i >= k_hi) break;
+      const __nv_bfloat162 w01 = *reinterpret_cast<const __nv_bfloat162*>(&wv[i].x);
+      const __nv_bfloat162 w23 = *reinterpret_cast<const __nv_bfloat162*>(&wv[i].y);
+      const float w[4] = {__low2float(w01), __high2float(w01), __low2float(w23), __high2float(w23)};
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    if (k_lo + i >= k_hi) break;
-    const __nv_bfloat162 w01 = *reinterpret_cast<const __nv_bfloat162*>(&wv[i].x);
-    const __nv_bfloat162 w23 = *reinterpret_cast<const __nv_bfloat162*>(&wv[i].y);
-    const float w[4] = {__low2float(w01), __high2float(w01), __low2float(w23), __high2float(w23)};
+      for (int bi = 0; bi < kAbsorbB; ++bi) {
+        const float qk = sq[bi][k0 + i];
 #pragma unroll
-    for (int bi = 0; bi < kAbsorbB; ++bi) {
-      const float qk = sq[bi][k_lo + i];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) acc[bi][j] = fmaf(qk, w[j], acc[bi][j]);
+        for (int j = 0; j < 4; ++j) acc[bi][j] = fmaf(qk, w[j], acc[bi][j]);
+      }
     }
   }
 #pragma unroll
@@ -248,8 +260,6 @@ __global__ void __launch_bounds__(192, 1) decode_attn_kernel(const __grid_consta
   volatile int* abort_flag = &sm->abort;
 
   const int g = blockIdx.x, hg = blockIdx.y;
-  const int seg_lo = a.cta_first_seg[g], seg_hi = a.cta_first_seg[g + 1];
-  if (seg_lo >= seg_hi) return;   // uniform: no work for this CTA
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int heads_valid = min(HG, a.H - hg * HG);
 
@@ -278,6 +288,10 @@ __global__ void __launch_bounds__(192, 1) decode_attn_kernel(const __grid_consta
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (threadIdx.x == 0) griddep_launch_dependents();
+  griddep_wait();   // the plan, the absorbed queries and the cache rows come from earlier kernels
+  const int seg_lo = a.cta_first_seg[g];
+  const int seg_hi = (seg_lo < a.cta_first_seg[g + 1]) ? a.cta_first_seg[g + 1] : seg_lo;   // empty: no work
   const uint32_t tmem = sm->tmem;
   const uint32_t tS = tmem;          // S^T: HG columns
   const uint32_t tO = tmem + HG;     // O^T: kNcBox/2 chunks of HG columns
@@ -586,6 +600,8 @@ __global__ void __launch_bounds__(192, 1) decode_attn_kernel(const __grid_consta
 //    its epilogue). Block (0, 0) also clears that GEMM's split-K tickets.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(128) decode_merge_kernel(DecodeArgs a) {
+  if (threadIdx.x == 0) griddep_launch_dependents();
+  griddep_wait();
   const int h = blockIdx.x, b = blockIdx.y;
   const int hg = h / a.HG, hl = h % a.HG;
   if (h == 0 && b == 0)
@@ -654,17 +670,16 @@ static cudaError_t launch_attn(const DecodeArgs& a, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
   prof_begin(st, "decode_attn");
-  k<<<dim3(a.G, a.n_hg), 192, C::kSmem, st>>>(a);
+  e = launch_pdl(k, dim3(a.G, a.n_hg), dim3(192), C::kSmem, st, 1, a);
   prof_end(st);
-  return cudaGetLastError();
+  return e;
 }
 
 cudaError_t launch_decode_bf16(DecodeArgs& a, cudaStream_t st) {
   const int n_absorb = a.H * ((a.B + kAbsorbB - 1) / kAbsorbB) * (a.d_c / kAbsorbCols);
   prof_begin(st, "decode_absorb_plan");
-  decode_absorb_plan_kernel<<<n_absorb + 1, 256, 0, st>>>(a);
+  cudaError_t e = launch_pdl(decode_absorb_plan_kernel, dim3(n_absorb + 1), dim3(256), 0, st, 1, a);
   prof_end(st);
-  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int nbox = (a.d_c + a.d_rope) / 64;
   switch (a.HG * 16 + nbox) {
@@ -678,9 +693,9 @@ cudaError_t launch_decode_bf16(DecodeArgs& a, cudaStream_t st) {
   }
   if (e != cudaSuccess) return e;
   prof_begin(st, "decode_merge");
-  decode_merge_kernel<<<dim3(a.H, a.B), 128, 0, st>>>(a);
+  e = launch_pdl(decode_merge_kernel, dim3(a.H, a.B), dim3(128), 0, st, 1, a);
   prof_end(st);
-  return cudaGetLastError();
+  return e;
 }
 
 }  // namespace gmla

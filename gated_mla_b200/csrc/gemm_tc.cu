@@ -88,6 +88,7 @@ __global__ void __launch_bounds__(192, 1) gemm_bf16_tc_kernel(const __grid_const
   int64_t* tok_row = reinterpret_cast<int64_t*>(smem + C::kStages * C::kStageBytes + 256);
   int* tok_pos = reinterpret_cast<int*>(tok_row + (kSwap ? BN : 1));
 
+  if (a.row_mode == 1) griddep_wait();   // the tile reads the sequence offsets
   GemmTile tile;
   if (!gemm_tile<BN, kSwap>(a, tile)) return;   // uniform across the block
 
@@ -126,6 +127,7 @@ __global__ void __launch_bounds__(192, 1) gemm_bf16_tc_kernel(const __grid_const
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (threadIdx.x == 0) griddep_launch_dependents();
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
@@ -135,6 +137,18 @@ __global__ void __launch_bounds__(192, 1) gemm_bf16_tc_kernel(const __grid_const
       tma_prefetch_desc(wmap);
       const uint64_t pol_w = l2_evict_normal();
       const uint64_t pol_x = l2_evict_last();
+      // Weight tiles are never written by a kernel: those of the first stages
+      // are requested before waiting for the kernel that produces the activations.
+      const int pre = min(num_kb, C::kStages);
+      for (int kb = 0; kb < pre; ++kb) {
+        uint8_t* sa = smem + kb * C::kStageBytes;
+        mbar_arrive_expect_tx(&full[kb], C::kStageBytes);
+        if (kSwap)
+          tma_load_2d(wmap, &full[kb], sa, (kb_begin + kb) * 64, tile.wrow0, pol_w);
+        else
+          tma_load_2d(wmap, &full[kb], sa + C::kABytes, kb * 64, tile.wrow0, pol_w);
+      }
+      griddep_wait();
       int issued = 0;
       for (int kb = 0; kb < num_kb; ++kb) {
         const int st = kb % C::kStages;
@@ -143,16 +157,17 @@ __global__ void __launch_bounds__(192, 1) gemm_bf16_tc_kernel(const __grid_const
           break;
         uint8_t* sa = smem + st * C::kStageBytes;
         uint8_t* sb = sa + C::kABytes;
-        mbar_arrive_expect_tx(&full[st], C::kStageBytes);
+        if (kb >= pre) mbar_arrive_expect_tx(&full[st], C::kStageBytes);
         if (kSwap) {
-          tma_load_2d(wmap, &full[st], sa, (kb_begin + kb) * 64, tile.wrow0, pol_w);
+          if (kb >= pre) tma_load_2d(wmap, &full[st], sa, (kb_begin + kb) * 64, tile.wrow0, pol_w);
           tma_load_2d(&a.act, &full[st], sb, (kb_begin + kb) * 64, tile.act_row0, pol_x);
         } else {
           tma_load_2d(&a.act, &full[st], sa, kb * 64, tile.act_row0, pol_x);
-          tma_load_2d(wmap, &full[st], sb, kb * 64, tile.wrow0, pol_w);
+          if (kb >= pre) tma_load_2d(wmap, &full[st], sb, kb * 64, tile.wrow0, pol_w);
         }
         ++issued;
       }
+      if (issued < pre) issued = pre;   // stages armed and partly loaded before the wait
       if (*abort_flag) {   // let copies still in flight land before the block exits
         for (int kb = max(0, issued - C::kStages); kb < issued; ++kb)
           mbar_drain(&full[kb % C::kStages], (kb / C::kStages) & 1);
@@ -189,6 +204,7 @@ __global__ void __launch_bounds__(192, 1) gemm_bf16_tc_kernel(const __grid_const
     // epilogue warps 2..5 -> TMEM lane quarter (warp % 4)
     const int q = warp & 3;
     const int r = q * 32 + lane;            // accumulator row of this thread
+    griddep_wait();                         // before reading positions or writing outputs
     // Split-K epilogues meet at named barrier 2; a failed wait still walks the
     // same barriers (with its stores skipped) so the four warps stay in step.
     const bool acc_ok = mbar_wait(acc_full, 0, abort_flag, a.status);
@@ -407,25 +423,8 @@ static cudaError_t launch_one(const GemmArgs& a, dim3 grid, cudaStream_t st, con
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   prof_begin(st, name);
-  if (kSwap && a.splits > 1) {
-    // the K splits of one tile run as a cluster along z
-    cudaLaunchConfig_t cfg{};
-    cfg.gridDim = grid;
-    cfg.blockDim = dim3(192);
-    cfg.dynamicSmemBytes = C::kSmemBytes;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 1;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = a.splits;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, k, a);
-  } else {
-    k<<<grid, 192, C::kSmemBytes, st>>>(a);
-    e = cudaGetLastError();
-  }
+  // the K splits of one tile (swap orientation) run as a cluster along z
+  e = launch_pdl(k, grid, dim3(192), C::kSmemBytes, st, (kSwap && a.splits > 1) ? a.splits : 1, a);
   prof_end(st);
   return e;
 }

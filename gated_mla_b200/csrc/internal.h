@@ -9,6 +9,35 @@
 
 namespace gmla {
 
+// Launches `kernel` with programmatic stream serialization: it may begin
+// while the previous kernel of the stream is still running, and calls
+// griddep_wait() before it touches data another kernel reads or writes. With
+// cluster_z > 1 the blocks form clusters of that size along z.
+template <typename Args>
+inline cudaError_t launch_pdl(void (*kernel)(Args), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              int cluster_z, const Args& args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  if (cluster_z > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = 1;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = static_cast<unsigned>(cluster_z);
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kernel, args);
+}
+
 // ----- tcgen05 GEMM (gemm_tc.cu) -----
 cudaError_t launch_gemm_bf16(const GemmArgs& a, bool swap, int bn, int token_tiles, cudaStream_t st,
                              const char* name);

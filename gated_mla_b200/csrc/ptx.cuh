@@ -170,6 +170,20 @@ __device__ __forceinline__ uint64_t l2_evict_normal() {
 }
 
 // ---------------------------------------------------------------------------
+// programmatic dependent launch
+// ---------------------------------------------------------------------------
+// Lets the next kernel of the stream (launched with programmatic stream
+// serialization) begin once every block of this grid has signalled or ended.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+// Waits until the grids this one depends on have completed and their memory
+// operations are visible; returns at once for a kernel launched without the
+// programmatic attribute. Every thread that touches data another kernel
+// reads or writes calls it first.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// ---------------------------------------------------------------------------
 // thread-block clusters (distributed shared memory; no multicast loads)
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t cluster_ctarank() {
