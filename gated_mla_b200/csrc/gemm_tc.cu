@@ -239,6 +239,16 @@ __global__ void __launch_bounds__(192, 1) gemm_bf16_tc_kernel(const __grid_const
         const float fbias = (e.bias && f_ok) ? e.bias[f] : 0.f;
         const int gcol = e.gate ? f / e.gate_div : 0;
         auto store_chunk = [&](int c0, float (&x)[16]) {
+          // the gate logits of the 16 tokens, all requested before any store
+          // (the compiler cannot move them past stores that might alias)
+          float gl[16];
+          if (e.gate) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              gl[j] = (tok_row[c0 + j] >= 0 && f_ok)
+                          ? e.gate[static_cast<int64_t>(tile.tok0 + c0 + j) * e.gate_stride + gcol]
+                          : 0.f;
+          }
 #pragma unroll 4
           for (int j = 0; j < 16; ++j) {
             const int tl = c0 + j;
@@ -251,8 +261,7 @@ __global__ void __launch_bounds__(192, 1) gemm_bf16_tc_kernel(const __grid_const
             const int64_t row = tok_row[tl];
             if (row < 0 || !f_ok) continue;
             val += fbias;
-            if (e.gate)
-              val *= 1.f / (1.f + __expf(-e.gate[static_cast<int64_t>(tile.tok0 + tl) * e.gate_stride + gcol]));
+            if (e.gate) val *= 1.f / (1.f + __expf(-gl[j]));
             const int64_t off = row * e.row_stride + colpart;
             if (e.out_f32)
               static_cast<float*>(e.out)[off] = val;
@@ -372,19 +381,38 @@ __global__ void __launch_bounds__(192, 1) gemm_bf16_tc_kernel(const __grid_const
         const float fbias = (e.bias && f_ok) ? e.bias[f] : 0.f;
         const int gcol = e.gate ? f / e.gate_div : 0;
 #pragma unroll 1
-        for (int c = 0; c < own_cols; c += 4) {
-          float x[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int c = 0; c < own_cols; c += 16) {
+          const int nc = min(16, own_cols - c);   // a multiple of 4
+          // gate logits of these tokens, all requested before any store
+          float gl[16];
+          if (e.gate) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const int tl = col0 + c + j;
+              gl[j] = (j < nc && tok_row[tl] >= 0 && f_ok)
+                          ? e.gate[static_cast<int64_t>(tile.tok0 + tl) * e.gate_stride + gcol]
+                          : 0.f;
+            }
+          }
+          float x[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) x[j] = 0.f;
 #pragma unroll
           for (int z = 0; z < 8; ++z) {
             if (z >= a.splits) break;
-            const float4 u = *reinterpret_cast<const float4*>(recv + (z * 128 + r) * cpr + c);
-            x[0] += u.x;
-            x[1] += u.y;
-            x[2] += u.z;
-            x[3] += u.w;
+#pragma unroll
+            for (int j = 0; j < 16; j += 4) {
+              if (j >= nc) break;
+              const float4 u = *reinterpret_cast<const float4*>(recv + (z * 128 + r) * cpr + c + j);
+              x[j] += u.x;
+              x[j + 1] += u.y;
+              x[j + 2] += u.z;
+              x[j + 3] += u.w;
+            }
           }
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
+          for (int j = 0; j < 16; ++j) {
+            if (j >= nc) break;
             const int tl = col0 + c + j;
             float val = x[j];
             if (e.rope) {
@@ -395,8 +423,7 @@ __global__ void __launch_bounds__(192, 1) gemm_bf16_tc_kernel(const __grid_const
             const int64_t row = tok_row[tl];
             if (row < 0 || !f_ok || !got) continue;
             val += fbias;
-            if (e.gate)
-              val *= 1.f / (1.f + __expf(-e.gate[static_cast<int64_t>(tile.tok0 + tl) * e.gate_stride + gcol]));
+            if (e.gate) val *= 1.f / (1.f + __expf(-gl[j]));
             const int64_t off = row * e.row_stride + colpart;
             if (e.out_f32)
               static_cast<float*>(e.out)[off] = val;
