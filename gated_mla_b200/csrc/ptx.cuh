@@ -351,6 +351,59 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
 }
+// max of three (one instruction on sm_100)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+// Pairs of fp32 in one 64-bit register, for the paired fp32 instructions of sm_100.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
+  return d;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t fsub2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// 2^x for two values on the FMA pipes (for x <= 2^22): x = n + f with n the
+// nearest integer (adding 1.5 * 2^23 leaves n in the low mantissa bits) and
+// |f| <= 1/2; 2^f from a degree-3 polynomial whose coefficients were fitted
+// here for relative error on [-1/2, 1/2] (at most 7.5e-5 in fp32); n is then
+// added to the exponent field. Inputs below -125 are clamped, so results
+// under 2^-125 come out as about 2^-125.
+__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& y0, float& y1) {
+  const float kMagic = 12582912.f;   // 1.5 * 2^23
+  const uint64_t x = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const uint64_t t = fadd2(x, f2_pack(kMagic, kMagic));
+  const uint64_t f = fsub2(x, fsub2(t, f2_pack(kMagic, kMagic)));   // t - magic = n exactly
+  uint64_t p = ffma2(f2_pack(0.055171623826026917f, 0.055171623826026917f), f,
+                     f2_pack(0.2426111251115799f, 0.2426111251115799f));
+  p = ffma2(p, f, f2_pack(0.6932609677314758f, 0.6932609677314758f));
+  p = ffma2(p, f, f2_pack(0.9999280571937561f, 0.9999280571937561f));
+  float p0, p1, t0, t1;
+  f2_unpack(p, p0, p1);
+  f2_unpack(t, t0, t1);
+  y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
+
 // Order-preserving map float -> int32 for integer max reductions.
 __device__ __forceinline__ int float_to_ordered(float f) {
   int i = __float_as_int(f);
