@@ -43,7 +43,9 @@ sys.path.insert(0, ROOT)
 DECODE_METRIC = "Gated-MLA decode latent-cache GB/s (latent_project + decode + gate_out step)"
 PREFILL_METRIC = "Gated-MLA prefill TFLOP/s (latent_project + prefill + gate_out step, explicit-form FLOPs)"
 DEFAULT_WORKLOAD = "decode_b32"
-FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+# the pool's earlier measurement: HBM copy, bf16 GEMM burst, and the same GEMM
+# sustained under the 1 kW power cap (about 1.4 PFLOP/s near 1.3 GHz)
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
 
@@ -73,7 +75,9 @@ def peaks():
     if os.path.exists(p):
         with open(p) as f:
             d = json.load(f)
-        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]), "source": "measured"}
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
     return dict(FALLBACK_PEAKS, source="fallback")
 
 
@@ -475,8 +479,12 @@ def run_ours(args):
             kernel_ms["step"] = max_total_ms / K
         dom = max(per, key=lambda k: kernel_ms[k])
         achieved = per[dom] / (kernel_ms[dom] / 1e3) / 1e12
-        roof = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": pk["bf16_tflops"],
-                "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"], "peak_source": pk["source"] + " burst",
+        # the prefill step runs for seconds back to back under the power cap:
+        # the sustained bf16 figure is the denominator (the burst one is kept beside it)
+        roof = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": pk["bf16_tflops_sustained"],
+                "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops_sustained"],
+                "peak_source": pk["source"] + " sustained", "peak_burst": pk["bf16_tflops"],
+                "frac_of_burst": achieved / pk["bf16_tflops"],
                 "traffic": None, "launch_ms": kernel_ms[dom], "algorithmic_flops_per_launch": per[dom],
                 "per_kernel_tflops": {k: per[k] / (kernel_ms[k] / 1e3) / 1e12 for k in per}}
 

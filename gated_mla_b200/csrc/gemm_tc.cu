@@ -312,12 +312,27 @@ __global__ void __launch_bounds__(192, 1) gemm_bf16_tc_kernel(const __grid_const
               x[j + 1] = rope_rotate(x1, x0, true, pos, fi >> 1, e.block, a.log2_rope_base);
             }
           }
-          const bool vec = !e.out_f32 && !e.bias && !e.gate && (f0 + 16 <= seg_rows) && (f0 % e.block) + 16 <= e.block &&
-                           ((row * e.row_stride + (f0 / e.block) * (int64_t)e.block_stride + (f0 % e.block) +
-                             e.col_offset) % 8 == 0);
-          if (vec) {
-            const int64_t off = row * e.row_stride + static_cast<int64_t>(f0 / e.block) * e.block_stride +
+          const int64_t off16 = row * e.row_stride + static_cast<int64_t>(f0 / e.block) * e.block_stride +
                                 (f0 % e.block) + e.col_offset;
+          const bool whole = !e.gate && (f0 + 16 <= seg_rows) && (f0 % e.block) + 16 <= e.block;
+          const bool vec = whole && !e.out_f32 && !e.bias && off16 % 8 == 0;
+          const bool vec32 = whole && e.out_f32 && off16 % 4 == 0;   // fp32 rows (+ bias), 16-byte stores
+          if (vec32) {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(e.out) + off16);
+#pragma unroll
+            for (int j = 0; j < 16; j += 4) {
+              float4 o = make_float4(x[j], x[j + 1], x[j + 2], x[j + 3]);
+              if (e.bias) {
+                const float4 bb = __ldg(reinterpret_cast<const float4*>(e.bias + f0 + j));
+                o.x += bb.x;
+                o.y += bb.y;
+                o.z += bb.z;
+                o.w += bb.w;
+              }
+              dst[j >> 2] = o;
+            }
+          } else if (vec) {
+            const int64_t off = off16;
             uint4 p0, p1;
             p0.x = pack_bf16x2(x[0], x[1]);
             p0.y = pack_bf16x2(x[2], x[3]);
