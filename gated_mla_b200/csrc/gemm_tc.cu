@@ -43,9 +43,25 @@ struct GemmTile {
   int ntok;      // valid tokens in this tile
 };
 
+// Large-token orientation: blocks are taken in groups of kGroupT token tiles,
+// the token tile varying fastest, so that the blocks resident at once share
+// few weight tiles and few token tiles and both stay in L2 (the plain order
+// would stream every weight tile from HBM once per token tile).
+constexpr int kGroupT = 16;
+
 template <int BN, bool kSwap>
 __device__ __forceinline__ bool gemm_tile(const GemmArgs& a, GemmTile& t) {
-  const int wt = blockIdx.x;
+  int wt = blockIdx.x, tt = blockIdx.y;
+  if (!kSwap) {
+    const int nw = gridDim.x, nt = gridDim.y;
+    const int lin = blockIdx.y * nw + blockIdx.x;
+    const int group = lin / (kGroupT * nw);
+    const int first = group * kGroupT;
+    const int gsize = min(kGroupT, nt - first);
+    const int in = lin - group * kGroupT * nw;
+    tt = first + in % gsize;
+    wt = in / gsize;
+  }
   int s = 0;
   while (s + 1 < a.n_seg && wt >= a.seg_tile_begin[s + 1]) ++s;
   t.seg = s;
@@ -53,17 +69,17 @@ __device__ __forceinline__ bool gemm_tile(const GemmArgs& a, GemmTile& t) {
   constexpr int kTTile = kSwap ? BN : 128;
   t.wrow0 = (wt - a.seg_tile_begin[s]) * kWTile;
   if (a.row_mode == 0) {
-    t.tok0 = blockIdx.y * kTTile;
+    t.tok0 = tt * kTTile;
     t.act_row0 = t.tok0;
     t.ntok = min(kTTile, a.T - t.tok0);
   } else if (a.row_mode == 2) {
-    t.tok0 = blockIdx.y * kTTile;
+    t.tok0 = tt * kTTile;
     t.act_row0 = (a.seg_tile_begin[s] * kWTile + t.wrow0) / a.rows_per_group * a.act_group_stride + t.tok0;
     t.ntok = min(kTTile, a.T - t.tok0);
   } else {
     // prefill sequence tiles: token tile -> (sequence, offset)
-    const int b = blockIdx.y / a.tiles_per_seq;
-    const int t0 = (blockIdx.y % a.tiles_per_seq) * kTTile;
+    const int b = tt / a.tiles_per_seq;
+    const int t0 = (tt % a.tiles_per_seq) * kTTile;
     const int beg = a.cu_seqlens[b], len = a.cu_seqlens[b + 1] - beg;
     t.tok0 = beg + t0;
     t.act_row0 = b * a.act_seq_stride + t0;
