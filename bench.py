@@ -219,10 +219,12 @@ def oracle_sample(inp, seconds: float, start: int = 0):
     p = oracle.params(inp)
     t0 = time.perf_counter()
     if w.mode == "decode":
-        # units of (sequence, 8 heads); work = that share of the sequence's latent bytes
+        # units of (sequence, 8 heads), sequences in turn (wrapping around the
+        # batch) until the time budget is spent; work = that share of the
+        # sequence's latent bytes
         units, nbytes, b = 0, 0.0, start
         hc = min(8, w.n_heads)
-        while True:
+        while time.perf_counter() - t0 < seconds:
             seq = b % w.batch
             for h0 in range(0, w.n_heads, hc):
                 heads = list(range(h0, min(w.n_heads, h0 + hc)))
@@ -232,13 +234,19 @@ def oracle_sample(inp, seconds: float, start: int = 0):
                 if time.perf_counter() - t0 >= seconds:
                     break
             b += 1
-            if time.perf_counter() - t0 >= seconds or b - start >= w.batch:
-                break
         return nbytes, time.perf_counter() - t0, f"{units} (sequence, {hc}-head) units from {b - start} sequences"
-    S = min(int(inp["lengths"][0]), 512)
-    oracle.prefill(p, inp["x"][:S], [S])
-    flops = sum(prefill_flops(w, [S]).values())
-    return flops, time.perf_counter() - t0, f"prefill of the first {S} tokens of sequence 0"
+    # prefill: prompts of the first min(L, 512) tokens of successive sequences
+    # until the time budget is spent
+    flops, n, b = 0.0, 0, start
+    while time.perf_counter() - t0 < seconds:
+        seq = b % w.batch
+        off = int(sum(int(L) for L in inp["lengths"][:seq]))
+        S = min(int(inp["lengths"][seq]), 512)
+        oracle.prefill(p, inp["x"][off:off + S], [S])
+        flops += sum(prefill_flops(w, [S]).values())
+        n += 1
+        b += 1
+    return flops, time.perf_counter() - t0, f"{n} prefills of the first min(L, 512) tokens of successive sequences"
 
 
 def work_unit(w):
