@@ -1,9 +1,7 @@
 // noalloc.cu — gmla_decode_noalloc: gmla_decode without a caller-provided
 // workspace.
 //
-// Some callers cannot hand the library a device buffer: code that runs while
-// a CUDA graph is being captured (cudaMalloc is not allowed there and
-// cudaMallocAsync would tie the memory to the graph), inference engines and
+// Some callers cannot hand the library a device buffer: inference engines and
 // plugins whose device memory is owned by their own pool and who forbid
 // third-party allocations, and latency-critical loops that cannot pay for
 // cudaMalloc's implicit device synchronisation. For them this file keeps the
@@ -12,8 +10,8 @@
 //
 // The array is kScratchBytes long and every GPU that loads the library holds
 // it until the process exits. Every call shares it and it keeps the previous
-// call's contents, so calls whose kernels overlap on the GPU (different
-// streams, or graphs replayed concurrently) race on it; serialise them.
+// call's contents, so calls whose kernels overlap on the GPU (for example on
+// different streams) race on it; serialise them.
 #include <cuda_runtime.h>
 
 #include <mutex>

@@ -194,8 +194,7 @@ GMLA_API gmla_status gmla_gate_out(const gmla_config* cfg, const gmla_weights* w
 
 /* ---------------------------------------------------------------------------
  * gmla_decode_noalloc — gmla_decode for callers that cannot allocate device
- * memory: code running under CUDA graph capture (cudaMalloc is not allowed
- * there), engines and plugins whose device memory belongs to their own pool,
+ * memory: engines and plugins whose device memory belongs to their own pool,
  * and loops that cannot pay cudaMalloc's implicit synchronisation. The pages
  * have no counterpart to this call: it is a deployment convenience.
  * Same arguments and results as gmla_decode, minus the workspace: the scratch
@@ -203,8 +202,7 @@ GMLA_API gmla_status gmla_gate_out(const gmla_config* cfg, const gmla_weights* w
  * loads the library until the process exits. The call allocates nothing.
  *   - Batches whose gmla_decode_workspace_size() exceeds 16 MiB are rejected
  *     with GMLA_ERR_WORKSPACE (use gmla_decode with a workspace instead).
- *   - The first call on a device looks up the array's device address; make
- *     that first call before any stream capture.
+ *   - The first call on a device looks up the array's device address.
  *   - All calls share the array and it keeps the previous call's contents:
  *     calls whose kernels overlap on the GPU race on it, so serialise them.
  *   - Device-side faults are recorded in the shared array's status word,

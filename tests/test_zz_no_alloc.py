@@ -1,6 +1,6 @@
 """gmla_decode_noalloc: the decode call for callers that cannot allocate device
-memory (graph capture, engines with their own memory pools, loops that cannot
-afford cudaMalloc's synchronisation). It keeps its scratch in a static device
+memory (engines with their own memory pools, loops that cannot afford
+cudaMalloc's synchronisation). It keeps its scratch in a static device
 array inside the library; here it must reproduce gmla_decode, which uses a
 caller-provided workspace, on two calls in a row through the C ABI.
 
