@@ -219,7 +219,7 @@ __global__ void __launch_bounds__(256, 4) decode_absorb_plan_kernel(DecodeArgs a
 // 3. attention over the latent cache
 // ---------------------------------------------------------------------------
 struct DecSmem {
-  uint64_t full[12], empty[12];
+  uint64_t full[6], empty[6];   // per box pair of the ring
   uint64_t rope_full, rope_empty;
   uint64_t q_full, q_empty;
   uint64_t s_full, p_full, o_done, o_free, drain;
@@ -242,7 +242,8 @@ struct DecCfg {
   static constexpr int kRingMax = (kBudget - kFixed) / kBoxBytes;
   static constexpr int kRing = (kRingMax > 12 ? 12 : kRingMax) & ~1;   // even: box pairs never wrap
   static constexpr int kSmem = kRing * kBoxBytes + kFixed;
-  static constexpr int kTmemCols = (5 * HG <= 128) ? 128 : ((5 * HG <= 256) ? 256 : 512);
+  // two S^T buffers of HG columns, then O^T: kNcBox/2 chunks of HG columns
+  static constexpr int kTmemCols = (6 * HG <= 128) ? 128 : ((6 * HG <= 256) ? 256 : 512);
   static_assert(kRing >= kNcBox, "ring must hold one tile");
 };
 
@@ -263,8 +264,9 @@ __global__ void __launch_bounds__(192, 1) decode_attn_kernel(const __grid_consta
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int heads_valid = min(HG, a.H - hg * HG);
 
+  constexpr int NP = NR / 2;   // ring slots hold box pairs: one full and one empty barrier each
   if (threadIdx.x == 0) {
-    for (int i = 0; i < NR; ++i) {
+    for (int i = 0; i < NP; ++i) {
       mbar_init(&sm->full[i], 1);
       mbar_init(&sm->empty[i], 1);
     }
@@ -293,8 +295,8 @@ __global__ void __launch_bounds__(192, 1) decode_attn_kernel(const __grid_consta
   const int seg_lo = a.cta_first_seg[g];
   const int seg_hi = (seg_lo < a.cta_first_seg[g + 1]) ? a.cta_first_seg[g + 1] : seg_lo;   // empty: no work
   const uint32_t tmem = sm->tmem;
-  const uint32_t tS = tmem;          // S^T: HG columns
-  const uint32_t tO = tmem + HG;     // O^T: kNcBox/2 chunks of HG columns
+  // S^T of tile n in columns [(n & 1) HG, +HG); O^T from column 2 HG in kNcBox/2 chunks of HG
+  const uint32_t tO = tmem + 2 * HG;
 
   if (warp == 0) {
     // ------------------------------ TMA producer ------------------------------
@@ -309,7 +311,7 @@ __global__ void __launch_bounds__(192, 1) decode_attn_kernel(const __grid_consta
     const uint64_t pol_q = l2_evict_last();
     const bool paged = a.cache.paged != 0;
     const int ps = paged ? a.cache.page_size : kTileTok;
-    uint32_t nbox = 0, nrope = 0, nq = 0;
+    uint32_t npair = 0, nrope = 0, nq = 0;
     bool ok = true;
     for (int si = seg_lo; si < seg_hi && ok; ++si) {
       const int4 sg = a.seg_info[si];
@@ -335,23 +337,25 @@ __global__ void __launch_bounds__(192, 1) decode_attn_kernel(const __grid_consta
           page = a.cache.block_table[static_cast<int64_t>(b) * a.cache.max_pages_per_seq + (tok0 + lane * ps) / ps];
         const uint32_t tx = ps >= kTileTok ? kBoxBytes : nchunk * ps * 128;
         for (int j = 0; j < NBOX; ++j) {
+          // ring boxes go in pairs (one barrier for both); the RoPE box has its own slot
           const bool ring_box = j < kNcBox;
-          const uint32_t slot = nbox % NR;
-          uint64_t* bar = ring_box ? &sm->full[slot] : &sm->rope_full;
-          uint8_t* dst = ring_box ? ring + slot * kBoxBytes : rope_slot;
+          const uint32_t pslot = npair % NP;
+          uint64_t* bar = ring_box ? &sm->full[pslot] : &sm->rope_full;
+          uint8_t* dst = ring_box ? ring + (pslot * 2 + (j & 1)) * kBoxBytes : rope_slot;
           if (lane == 0) {
-            if (ring_box) {
-              if (nbox >= static_cast<uint32_t>(NR) &&
-                  !mbar_wait(&sm->empty[slot], ((nbox / NR) & 1) ^ 1, abort_flag, a.status))
+            if (!ring_box) {
+              if (nrope > 0 && !mbar_wait(&sm->rope_empty, (nrope - 1) & 1, abort_flag, a.status)) ok = false;
+              if (ok) mbar_arrive_expect_tx(bar, tx);
+            } else if ((j & 1) == 0) {
+              if (npair >= static_cast<uint32_t>(NP) &&
+                  !mbar_wait(&sm->empty[pslot], ((npair / NP) & 1) ^ 1, abort_flag, a.status))
                 ok = false;
-            } else if (nrope > 0 && !mbar_wait(&sm->rope_empty, (nrope - 1) & 1, abort_flag, a.status)) {
-              ok = false;
+              if (ok) mbar_arrive_expect_tx(bar, 2 * tx);
             }
-            if (ok) mbar_arrive_expect_tx(bar, tx);
           }
           ok = __shfl_sync(0xffffffffu, ok, 0);
           if (!ok) break;
-          if (ring_box) ++nbox; else ++nrope;
+          if (!ring_box) ++nrope; else if (j & 1) ++npair;
           if (!paged) {
             if (lane == 0) tma_load_2d(&a.cache_map, bar, dst, j * 64, b * a.cache.capacity + tok0, pol_c);
           } else if (ps >= kTileTok) {
@@ -363,44 +367,68 @@ __global__ void __launch_bounds__(192, 1) decode_attn_kernel(const __grid_consta
       }
     }
     if (lane == 0 && *abort_flag) {   // let issued copies land before the block exits
-      for (uint32_t c = nbox > static_cast<uint32_t>(NR) ? nbox - NR : 0; c < nbox; ++c)
-        mbar_drain(&sm->full[c % NR], (c / NR) & 1);
+      for (uint32_t c = npair > static_cast<uint32_t>(NP) ? npair - NP : 0; c < npair; ++c)
+        mbar_drain(&sm->full[c % NP], (c / NP) & 1);
       if (nrope) mbar_drain(&sm->rope_full, (nrope - 1) & 1);
       if (nq) mbar_drain(&sm->q_full, (nq - 1) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------ MMA issuer ------------------------------
+    // Per tile: the score MMAs (S^T = C Q^T) of the pairs not yet issued, then
+    // while the softmax works on this tile, the first pairs of the next tile
+    // (into the other S^T buffer) if their boxes have landed, then the weighted
+    // sum O^T += C^T P^T once P is ready, which frees the tile's pairs.
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16_f32(128, HG, false, false);
       constexpr uint32_t idO = idesc_bf16_f32(128, HG, true, false);
       const uint32_t ring_a = smem_u32(ring), rope_a = smem_u32(rope_slot), q_a = smem_u32(qs),
                      p_a = smem_u32(pbuf);
-      uint32_t nbox = 0, nrope = 0, ntile = 0, nseg = 0;
+      uint32_t npair = 0, nrope = 0, ntile = 0, nseg = 0;
+      int early = 0;   // pairs of this tile whose score MMAs were issued during the previous tile
       bool ok = true;
+      auto s_pair = [&](uint32_t c, int p, uint32_t tSb) {   // ring pair c holds boxes 2p, 2p+1
+        const uint32_t sa = ring_a + (c % NP) * 2 * kBoxBytes;
+#pragma unroll
+        for (int b2 = 0; b2 < 2; ++b2) {
+          const int j = 2 * p + b2;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16(tSb, sdesc_sw128(sa + b2 * kBoxBytes + kk * 32, 16, 1024),
+                      sdesc_sw128(q_a + j * HG * 128 + kk * 32, 16, 1024), idS, (j | kk) != 0);
+        }
+      };
       for (int si = seg_lo; si < seg_hi && ok; ++si, ++nseg) {
         const int4 sg = a.seg_info[si];
         if (!mbar_wait(&sm->q_full, nseg & 1, abort_flag, a.status)) { ok = false; break; }
         for (int t = sg.y; t < sg.z; ++t, ++ntile) {
-          // S^T = C Q^T
-          for (int j = 0; j < NBOX; ++j) {
-            uint32_t sa;
-            if (j < kNcBox) {
-              const uint32_t c = nbox + j, slot = c % NR;
-              if (!mbar_wait(&sm->full[slot], (c / NR) & 1, abort_flag, a.status)) { ok = false; break; }
-              sa = ring_a + slot * kBoxBytes;
-            } else {
-              if (!mbar_wait(&sm->rope_full, nrope & 1, abort_flag, a.status)) { ok = false; break; }
-              sa = rope_a;
-            }
-            tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              umma_bf16(tS, sdesc_sw128(sa + kk * 32, 16, 1024),
-                        sdesc_sw128(q_a + j * HG * 128 + kk * 32, 16, 1024), idS, (j | kk) != 0);
+          const uint32_t tSb = tmem + (ntile & 1) * HG;
+          for (int p = early; p < kNcBox / 2; ++p) {
+            const uint32_t c = npair + p;
+            if (!mbar_wait(&sm->full[c % NP], (c / NP) & 1, abort_flag, a.status)) { ok = false; break; }
+            s_pair(c, p, tSb);   // boxes are ordered by their TMA barrier: no tcgen05 fence needed
           }
           if (!ok) break;
+          if (C::kRope) {
+            if (!mbar_wait(&sm->rope_full, nrope & 1, abort_flag, a.status)) { ok = false; break; }
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              umma_bf16(tSb, sdesc_sw128(rope_a + kk * 32, 16, 1024),
+                        sdesc_sw128(q_a + kNcBox * HG * 128 + kk * 32, 16, 1024), idS, 1u);
+          }
           if (t + 1 == sg.z) umma_commit(&sm->q_empty);
           umma_commit(&sm->s_full);
+          // the next tile of this segment: its first pairs, if they have landed (a
+          // non-blocking probe, so a late pair never holds up this tile's weighted sum)
+          early = 0;
+          if (t + 1 < sg.z) {
+            const uint32_t tSn = tmem + ((ntile + 1) & 1) * HG;
+            for (int p = 0; p < 2; ++p) {
+              const uint32_t c = npair + kNcBox / 2 + p;
+              if (!mbar_test(&sm->full[c % NP], (c / NP) & 1)) break;
+              s_pair(c, p, tSn);
+              ++early;
+            }
+          }
           // wait for P, then O^T += C^T P^T
           if (!mbar_wait(&sm->p_full, ntile & 1, abort_flag, a.status)) { ok = false; break; }
           const bool first = (t == sg.y);
@@ -408,19 +436,18 @@ __global__ void __launch_bounds__(192, 1) decode_attn_kernel(const __grid_consta
           tc_fence_after();
 #pragma unroll 1
           for (int mc = 0; mc < kNcBox / 2; ++mc) {
-            const uint32_t c0 = nbox + 2 * mc, slot0 = c0 % NR;
-            const uint32_t sa = ring_a + slot0 * kBoxBytes;
+            const uint32_t pslot = (npair + mc) % NP;
+            const uint32_t sa = ring_a + pslot * 2 * kBoxBytes;
 #pragma unroll
             for (int kk = 0; kk < kTileTok / 16; ++kk) {
               const uint64_t ad = sdesc_sw128(sa + kk * 2048, kBoxBytes, 1024);
               const uint64_t bd = sdesc_sw128(p_a + (kk >> 2) * (HG * 128) + (kk & 3) * 32, 16, 1024);
               umma_bf16(tO + mc * HG, ad, bd, idO, (!first || kk > 0) ? 1u : 0u);
             }
-            umma_commit(&sm->empty[slot0]);
-            umma_commit(&sm->empty[slot0 + 1]);
+            umma_commit(&sm->empty[pslot]);
           }
           if (C::kRope) umma_commit(&sm->rope_empty);
-          nbox += kNcBox;
+          npair += kNcBox / 2;
           if (C::kRope) ++nrope;
         }
         if (!ok) break;
@@ -460,7 +487,7 @@ __global__ void __launch_bounds__(192, 1) decode_attn_kernel(const __grid_consta
 #pragma unroll
         for (int c = 0; c < HG; c += 16) {
           uint32_t v[16];
-          tmem_ld16(tS + lane_off + c, v);
+          tmem_ld16(tmem + (ntile & 1) * HG + lane_off + c, v);
           tmem_ld_wait();
 #pragma unroll
           for (int j = 0; j < 16; ++j) s[c + j] = __uint_as_float(v[j]);

@@ -199,7 +199,8 @@ __global__ void __launch_bounds__(192, 1) gemm_bf16_tc_kernel(const __grid_const
           ok = false;
           break;
         }
-        tc_fence_after();
+        // the stage is ordered by its TMA barrier; a tcgen05 fence per stage would
+        // drain the tensor pipe between k-blocks
         const uint32_t sa = smem_u32(smem + st * C::kStageBytes);
         const uint32_t sb = sa + C::kABytes;
 #pragma unroll

@@ -163,8 +163,7 @@ __global__ void __launch_bounds__(576, 1) prefill_attn_kernel(const __grid_const
               break;
             }
             next_loaded = true;
-            tc_fence_after();
-            issue_s(0, j + 1);
+            issue_s(0, j + 1);   // K tile ordered by its TMA barrier; TMEM reuse by the P_A wait
           }
         }
         if (hasB) {
@@ -179,8 +178,7 @@ __global__ void __launch_bounds__(576, 1) prefill_attn_kernel(const __grid_const
             ok = false;
             break;
           }
-          tc_fence_after();
-          issue_s(1, j + 1);
+          issue_s(1, j + 1);   // TMEM reuse ordered by the P_B wait above
         }
       }
       if (ok) {
