@@ -386,15 +386,19 @@ __global__ void __launch_bounds__(192, 1) decode_attn_kernel(const __grid_consta
       uint32_t npair = 0, nrope = 0, ntile = 0, nseg = 0;
       int early = 0;   // pairs of this tile whose score MMAs were issued during the previous tile
       bool ok = true;
+      // Descriptors are built once; an operand's descriptor is the base one plus its
+      // byte offset / 16 (the start-address field cannot carry: shared addresses < 256 KB).
+      const uint64_t dRing = sdesc_sw128(ring_a, 16, 1024), dQ = sdesc_sw128(q_a, 16, 1024);
+      const uint64_t dRingMN = sdesc_sw128(ring_a, kBoxBytes, 1024), dP = sdesc_sw128(p_a, 16, 1024);
       auto s_pair = [&](uint32_t c, int p, uint32_t tSb) {   // ring pair c holds boxes 2p, 2p+1
-        const uint32_t sa = ring_a + (c % NP) * 2 * kBoxBytes;
+        const uint64_t da = dRing + (c % NP) * (2 * kBoxBytes / 16);
+        const uint64_t db = dQ + p * (2 * HG * 128 / 16);
 #pragma unroll
         for (int b2 = 0; b2 < 2; ++b2) {
-          const int j = 2 * p + b2;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            umma_bf16(tSb, sdesc_sw128(sa + b2 * kBoxBytes + kk * 32, 16, 1024),
-                      sdesc_sw128(q_a + j * HG * 128 + kk * 32, 16, 1024), idS, (j | kk) != 0);
+            umma_bf16(tSb, da + (b2 * kBoxBytes + kk * 32) / 16, db + (b2 * HG * 128 + kk * 32) / 16, idS,
+                      (p | b2 | kk) != 0);
         }
       };
       for (int si = seg_lo; si < seg_hi && ok; ++si, ++nseg) {
@@ -412,8 +416,8 @@ __global__ void __launch_bounds__(192, 1) decode_attn_kernel(const __grid_consta
             if (!mbar_wait(&sm->rope_full, nrope & 1, abort_flag, a.status)) { ok = false; break; }
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-              umma_bf16(tSb, sdesc_sw128(rope_a + kk * 32, 16, 1024),
-                        sdesc_sw128(q_a + kNcBox * HG * 128 + kk * 32, 16, 1024), idS, 1u);
+              umma_bf16(tSb, sdesc_sw128(rope_a + kk * 32, 16, 1024), dQ + (kNcBox * HG * 128 + kk * 32) / 16, idS,
+                        1u);
           }
           if (t + 1 == sg.z) umma_commit(&sm->q_empty);
           umma_commit(&sm->s_full);
@@ -437,13 +441,11 @@ __global__ void __launch_bounds__(192, 1) decode_attn_kernel(const __grid_consta
 #pragma unroll 1
           for (int mc = 0; mc < kNcBox / 2; ++mc) {
             const uint32_t pslot = (npair + mc) % NP;
-            const uint32_t sa = ring_a + pslot * 2 * kBoxBytes;
+            const uint64_t da = dRingMN + pslot * (2 * kBoxBytes / 16);
 #pragma unroll
-            for (int kk = 0; kk < kTileTok / 16; ++kk) {
-              const uint64_t ad = sdesc_sw128(sa + kk * 2048, kBoxBytes, 1024);
-              const uint64_t bd = sdesc_sw128(p_a + (kk >> 2) * (HG * 128) + (kk & 3) * 32, 16, 1024);
-              umma_bf16(tO + mc * HG, ad, bd, idO, (!first || kk > 0) ? 1u : 0u);
-            }
+            for (int kk = 0; kk < kTileTok / 16; ++kk)
+              umma_bf16(tO + mc * HG, da + kk * (2048 / 16), dP + ((kk >> 2) * (HG * 128) + (kk & 3) * 32) / 16, idO,
+                        (!first || kk > 0) ? 1u : 0u);
             umma_commit(&sm->empty[pslot]);
           }
           if (C::kRope) umma_commit(&sm->rope_empty);
