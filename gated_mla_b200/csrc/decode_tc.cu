@@ -228,11 +228,14 @@ struct DecSmem {
   int vote[2];
   int red[2][4][64];
   float lred[4][64];
+  float mfin[64];
 };
 
 template <int HG, int NBOX>
 struct DecCfg {
   static constexpr bool kRope = NBOX > kNcBox;
+  static constexpr int kSG = HG >= 32 ? 2 : 1;              // softmax warp groups (head slices)
+  static constexpr int kThreads = 64 + 128 * kSG;
   static constexpr int kQBytes = NBOX * HG * 128;          // absorbed queries, NBOX boxes of [HG x 64]
   static constexpr int kPBytes = kRope ? 0 : HG * 256;     // P [HG x 128] (K-major, 2 blocks); rope slot otherwise
   static constexpr int kRopeBytes = kRope ? kBoxBytes : 0;
@@ -248,7 +251,7 @@ struct DecCfg {
 };
 
 template <int HG, int NBOX>
-__global__ void __launch_bounds__(192, 1) decode_attn_kernel(const __grid_constant__ DecodeArgs a) {
+__global__ void __launch_bounds__(64 + 128 * (HG >= 32 ? 2 : 1), 1) decode_attn_kernel(const __grid_constant__ DecodeArgs a) {
   using C = DecCfg<HG, NBOX>;
   constexpr int NR = C::kRing;
   extern __shared__ uint8_t smem_raw[];
@@ -275,9 +278,9 @@ __global__ void __launch_bounds__(192, 1) decode_attn_kernel(const __grid_consta
     mbar_init(&sm->q_full, 1);
     mbar_init(&sm->q_empty, 1);
     mbar_init(&sm->s_full, 1);
-    mbar_init(&sm->p_full, 128);
+    mbar_init(&sm->p_full, 128 * C::kSG);
     mbar_init(&sm->o_done, 1);
-    mbar_init(&sm->o_free, 128);
+    mbar_init(&sm->o_free, 128 * C::kSG);
     mbar_init(&sm->drain, 1);
     sm->abort = 0;
     sm->vote[0] = sm->vote[1] = 0;
@@ -462,22 +465,26 @@ __global__ void __launch_bounds__(192, 1) decode_attn_kernel(const __grid_consta
     }
   } else {
     // ------------------------------ softmax warps ------------------------------
+    // 4 * SG warps: warp w reads TMEM lane quarter w % 4 (one token row per
+    // thread) and owns heads [h0, h0 + HT) of the head group.
+    constexpr int SG = C::kSG, HT = HG / SG;
     const int q4 = warp & 3;
+    const int h0 = SG == 1 ? 0 : ((warp - 2) >> 2) * HT;
     const int row = q4 * 32 + lane;                      // token row of the tile / latent row of a chunk
     const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
-    const int ltid = threadIdx.x - 64;                   // 0..127
+    const int ltid = threadIdx.x - 64;                   // 0 .. 128 SG - 1
     const float NEG_INF = -__int_as_float(0x7f800000);
-    // The four softmax warps meet at named barrier 1. After a failed wait a
-    // warp keeps walking the same loops (skipping the waits) so every warp
-    // executes the same sequence of barriers and the block can exit.
+    // The softmax warps meet at named barrier 1. After a failed wait a warp
+    // keeps walking the same loops (skipping the waits) so every warp executes
+    // the same sequence of barriers and the block can exit.
     uint32_t nbox = 0, ntile = 0, nseg = 0;
     bool ok = true;
     for (int si = seg_lo; si < seg_hi; ++si, ++nseg) {
       const int4 sg = a.seg_info[si];
       const int L = a.seq_lens[sg.x];
-      float m[HG], lsum[HG];
+      float m[HT], lsum[HT];
 #pragma unroll
-      for (int h = 0; h < HG; ++h) {
+      for (int h = 0; h < HT; ++h) {
         m[h] = NEG_INF;
         lsum[h] = 0.f;
       }
@@ -485,11 +492,11 @@ __global__ void __launch_bounds__(192, 1) decode_attn_kernel(const __grid_consta
         const bool first = (t == sg.y);
         ok = ok && mbar_wait(&sm->s_full, ntile & 1, abort_flag, a.status);
         tc_fence_after();
-        float s[HG];
+        float s[HT];
 #pragma unroll
-        for (int c = 0; c < HG; c += 16) {
+        for (int c = 0; c < HT; c += 16) {
           uint32_t v[16];
-          tmem_ld16(tmem + (ntile & 1) * HG + lane_off + c, v);
+          tmem_ld16(tmem + (ntile & 1) * HG + lane_off + h0 + c, v);
           tmem_ld_wait();
 #pragma unroll
           for (int j = 0; j < 16; ++j) s[c + j] = __uint_as_float(v[j]);
@@ -498,31 +505,31 @@ __global__ void __launch_bounds__(192, 1) decode_attn_kernel(const __grid_consta
         const bool rv = row < valid;
         bool need = first;
 #pragma unroll
-        for (int h = 0; h < HG; ++h) {
+        for (int h = 0; h < HT; ++h) {
           if (!rv) s[h] = NEG_INF;
           need |= s[h] > m[h] + 8.f;
         }
-        // block-wide vote among the 128 softmax threads
+        // block-wide vote among the softmax threads
         const int par = ntile & 1;
         if (__any_sync(0xffffffffu, need) && lane == 0) atomicOr(&sm->vote[par], 1);
-        asm volatile("bar.sync 1, 128;" ::: "memory");
+        asm volatile("bar.sync 1, %0;" ::"n"(128 * SG) : "memory");
         const bool need_all = sm->vote[par] != 0;
         if (ltid == 0) sm->vote[par ^ 1] = 0;
         if (need_all) {
 #pragma unroll
-          for (int h = 0; h < HG; ++h) {
+          for (int h = 0; h < HT; ++h) {
             const int k = __reduce_max_sync(0xffffffffu, float_to_ordered(s[h]));
-            if (lane == 0) sm->red[par][q4][h] = k;
+            if (lane == 0) sm->red[par][q4][h0 + h] = k;
           }
-          asm volatile("bar.sync 1, 128;" ::: "memory");
-          float alpha[HG];
+          asm volatile("bar.sync 1, %0;" ::"n"(128 * SG) : "memory");
+          float alpha[HT];
           bool rescale = false;
 #pragma unroll
-          for (int h = 0; h < HG; ++h) {
-            int k = sm->red[par][0][h];
-            k = max(k, sm->red[par][1][h]);
-            k = max(k, sm->red[par][2][h]);
-            k = max(k, sm->red[par][3][h]);
+          for (int h = 0; h < HT; ++h) {
+            int k = sm->red[par][0][h0 + h];
+            k = max(k, sm->red[par][1][h0 + h]);
+            k = max(k, sm->red[par][2][h0 + h]);
+            k = max(k, sm->red[par][3][h0 + h]);
             const float tmax = ordered_to_float(k);
             const float mn = fmaxf(m[h], tmax);
             alpha[h] = (m[h] == NEG_INF) ? 0.f : ex2_approx(m[h] - mn);
@@ -532,27 +539,28 @@ __global__ void __launch_bounds__(192, 1) decode_attn_kernel(const __grid_consta
           }
           if (rescale) {
             // O^T columns of head h scale by alpha[h] (O of the previous tile is complete:
-            // S of this tile was issued after it)
+            // S of this tile was committed after it)
 #pragma unroll 1
             for (int mc = 0; mc < kNcBox / 2; ++mc) {
 #pragma unroll
-              for (int c = 0; c < HG; c += 16) {
+              for (int c = 0; c < HT; c += 16) {
                 uint32_t v[16];
-                tmem_ld16(tO + lane_off + mc * HG + c, v);
+                tmem_ld16(tO + lane_off + mc * HG + h0 + c, v);
                 tmem_ld_wait();
 #pragma unroll
                 for (int j = 0; j < 16; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * alpha[c + j]);
-                tmem_st16(tO + lane_off + mc * HG + c, v);
+                tmem_st16(tO + lane_off + mc * HG + h0 + c, v);
               }
             }
             tmem_st_wait();
           }
         }
         // P = exp2(s - m), stored bf16 as P[h][token] (K-major B operand, 2 blocks of 64 tokens)
-        uint8_t* pb = pbuf + (row >> 6) * (HG * 128);
+        // (h0 is a multiple of 8, so the swizzle of row h0 + h is that of row h)
+        uint8_t* pb = pbuf + (row >> 6) * (HG * 128) + h0 * 128;
         const int pc = row & 63;
 #pragma unroll
-        for (int h = 0; h < HG; ++h) {
+        for (int h = 0; h < HT; ++h) {
           const float p = rv ? ex2_approx(s[h] - m[h]) : 0.f;
           lsum[h] += p;
           *reinterpret_cast<__nv_bfloat16*>(pb + sw128_offset(h, pc)) = __float2bfloat16_rn(p);
@@ -560,7 +568,7 @@ __global__ void __launch_bounds__(192, 1) decode_attn_kernel(const __grid_consta
         if (!rv) {
           // rows past the sequence end may hold anything: zero them so 0 * garbage cannot reach O
 #pragma unroll 1
-          for (int j = 0; j < kNcBox; ++j) {
+          for (int j = h0 / HT; j < kNcBox; j += SG) {
             uint8_t* box = ring + ((nbox + j) % NR) * kBoxBytes + row * 128;
 #pragma unroll
             for (int c = 0; c < 8; ++c) reinterpret_cast<uint4*>(box)[c] = make_uint4(0, 0, 0, 0);
@@ -574,22 +582,24 @@ __global__ void __launch_bounds__(192, 1) decode_attn_kernel(const __grid_consta
       // ---- segment end: write the partial (unnormalised O, running max m, sum l)
       ok = ok && mbar_wait(&sm->o_done, nseg & 1, abort_flag, a.status);
       tc_fence_after();
-      const int par = nseg & 1;
-      (void)par;
 #pragma unroll
-      for (int h = 0; h < HG; ++h) {
+      for (int h = 0; h < HT; ++h) {
         float v = lsum[h];
         for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        if (lane == 0) sm->lred[q4][h] = v;
+        if (lane == 0) sm->lred[q4][h0 + h] = v;
+        if (SG > 1 && lane == 0 && q4 == 0) sm->mfin[h0 + h] = m[h];   // the running max is the same in every row
       }
-      asm volatile("bar.sync 1, 128;" ::: "memory");
+      asm volatile("bar.sync 1, %0;" ::"n"(128 * SG) : "memory");
       const int64_t pbase = (static_cast<int64_t>(hg) * a.max_seg + si) * HG;
       if (ok && ltid < heads_valid) {
-        float l = 0.f;
-        float mh = NEG_INF;
+        float l = 0.f, mh = NEG_INF;
+        if (SG == 1) {   // every thread holds the running max of every head
 #pragma unroll
-        for (int h = 0; h < HG; ++h)
-          if (h == ltid) mh = m[h];
+          for (int h = 0; h < HT; ++h)
+            if (h == ltid) mh = m[h];
+        } else {
+          mh = sm->mfin[ltid];
+        }
         for (int w = 0; w < 4; ++w) l += sm->lred[w][ltid];
         a.ml_part[(pbase + ltid) * 2 + 0] = mh;
         a.ml_part[(pbase + ltid) * 2 + 1] = l;
@@ -597,19 +607,19 @@ __global__ void __launch_bounds__(192, 1) decode_attn_kernel(const __grid_consta
 #pragma unroll 1
       for (int mc = 0; mc < kNcBox / 2; ++mc) {
 #pragma unroll
-        for (int c = 0; c < HG; c += 16) {
+        for (int c = 0; c < HT; c += 16) {
           uint32_t v[16];
-          tmem_ld16(tO + lane_off + mc * HG + c, v);
+          tmem_ld16(tO + lane_off + mc * HG + h0 + c, v);
           tmem_ld_wait();
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            if (ok && c + j < heads_valid)
-              a.o_part[(pbase + c + j) * kDc + mc * 128 + row] = __uint_as_float(v[j]);
+            if (ok && h0 + c + j < heads_valid)
+              a.o_part[(pbase + h0 + c + j) * kDc + mc * 128 + row] = __uint_as_float(v[j]);
           }
         }
       }
       tc_fence_before();
-      asm volatile("bar.sync 1, 128;" ::: "memory");   // lred reuse
+      asm volatile("bar.sync 1, %0;" ::"n"(128 * SG) : "memory");   // lred / mfin reuse
       mbar_arrive(&sm->o_free);
     }
   }
@@ -699,7 +709,7 @@ static cudaError_t launch_attn(const DecodeArgs& a, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
   prof_begin(st, "decode_attn");
-  e = launch_pdl(k, dim3(a.G, a.n_hg), dim3(192), C::kSmem, st, 1, a);
+  e = launch_pdl(k, dim3(a.G, a.n_hg), dim3(C::kThreads), C::kSmem, st, 1, a);
   prof_end(st);
   return e;
 }
