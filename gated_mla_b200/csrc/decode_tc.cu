@@ -237,7 +237,10 @@ struct DecCfg {
   static constexpr int kSG = HG >= 32 ? 2 : 1;              // softmax warp groups (head slices)
   static constexpr int kThreads = 64 + 128 * kSG;
   static constexpr int kQBytes = NBOX * HG * 128;          // absorbed queries, NBOX boxes of [HG x 64]
-  static constexpr int kPBytes = kRope ? 0 : HG * 256;     // P [HG x 128] (K-major, 2 blocks); rope slot otherwise
+  static constexpr int kPBytes = kRope ? 0 : HG * 256;     // P [128 tokens x HG]; in the RoPE slot otherwise
+  // P is the MN-major B operand of O^T = C^T P^T: token rows of HG bf16 in
+  // swizzle atoms of 8 rows (HG 64: 128-byte rows, HG 32: 64, HG 16: 32)
+  static constexpr uint32_t kPLayout = HG == 64 ? 2u : (HG == 32 ? 4u : 6u);
   static constexpr int kRopeBytes = kRope ? kBoxBytes : 0;
   static constexpr int kSmemStruct = (static_cast<int>(sizeof(DecSmem)) + 127) & ~127;
   static constexpr int kFixed = kQBytes + kPBytes + kRopeBytes + kSmemStruct + 1024 /*align*/;
@@ -383,7 +386,7 @@ __global__ void __launch_bounds__(64 + 128 * (HG >= 32 ? 2 : 1), 1) decode_attn_
     // sum O^T += C^T P^T once P is ready, which frees the tile's pairs.
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16_f32(128, HG, false, false);
-      constexpr uint32_t idO = idesc_bf16_f32(128, HG, true, false);
+      constexpr uint32_t idO = idesc_bf16_f32(128, HG, true, true);
       const uint32_t ring_a = smem_u32(ring), rope_a = smem_u32(rope_slot), q_a = smem_u32(qs),
                      p_a = smem_u32(pbuf);
       uint32_t npair = 0, nrope = 0, ntile = 0, nseg = 0;
@@ -392,7 +395,8 @@ __global__ void __launch_bounds__(64 + 128 * (HG >= 32 ? 2 : 1), 1) decode_attn_
       // Descriptors are built once; an operand's descriptor is the base one plus its
       // byte offset / 16 (the start-address field cannot carry: shared addresses < 256 KB).
       const uint64_t dRing = sdesc_sw128(ring_a, 16, 1024), dQ = sdesc_sw128(q_a, 16, 1024);
-      const uint64_t dRingMN = sdesc_sw128(ring_a, kBoxBytes, 1024), dP = sdesc_sw128(p_a, 16, 1024);
+      const uint64_t dRingMN = sdesc_sw128(ring_a, kBoxBytes, 1024);
+      const uint64_t dP = sdesc_swz(p_a, kTileTok * HG * 2, 8 * HG * 2, C::kPLayout);   // one atom wide (N = HG)
       auto s_pair = [&](uint32_t c, int p, uint32_t tSb) {   // ring pair c holds boxes 2p, 2p+1
         const uint64_t da = dRing + (c % NP) * (2 * kBoxBytes / 16);
         const uint64_t db = dQ + p * (2 * HG * 128 / 16);
@@ -447,7 +451,7 @@ __global__ void __launch_bounds__(64 + 128 * (HG >= 32 ? 2 : 1), 1) decode_attn_
             const uint64_t da = dRingMN + pslot * (2 * kBoxBytes / 16);
 #pragma unroll
             for (int kk = 0; kk < kTileTok / 16; ++kk)
-              umma_bf16(tO + mc * HG, da + kk * (2048 / 16), dP + ((kk >> 2) * (HG * 128) + (kk & 3) * 32) / 16, idO,
+              umma_bf16(tO + mc * HG, da + kk * (2048 / 16), dP + kk * (16 * HG * 2 / 16), idO,
                         (!first || kk > 0) ? 1u : 0u);
             umma_commit(&sm->empty[pslot]);
           }
@@ -555,15 +559,23 @@ __global__ void __launch_bounds__(64 + 128 * (HG >= 32 ? 2 : 1), 1) decode_attn_
             tmem_st_wait();
           }
         }
-        // P = exp2(s - m), stored bf16 as P[h][token] (K-major B operand, 2 blocks of 64 tokens)
-        // (h0 is a multiple of 8, so the swizzle of row h0 + h is that of row h)
-        uint8_t* pb = pbuf + (row >> 6) * (HG * 128) + h0 * 128;
-        const int pc = row & 63;
+        // P = exp2(s - m) as bf16, this thread's token row of P[token][head]: 16-byte
+        // chunks of 8 heads, chunk index XOR the row bits of the swizzle atom
+        uint8_t* pb = pbuf + row * (HG * 2);
+        const int sw = HG == 64 ? (row & 7) : (HG == 32 ? ((row >> 1) & 3) : ((row >> 2) & 1));
 #pragma unroll
-        for (int h = 0; h < HT; ++h) {
-          const float p = rv ? ex2_approx(s[h] - m[h]) : 0.f;
-          lsum[h] += p;
-          *reinterpret_cast<__nv_bfloat16*>(pb + sw128_offset(h, pc)) = __float2bfloat16_rn(p);
+        for (int c = 0; c < HT; c += 8) {
+          uint32_t w[4];
+#pragma unroll
+          for (int k = 0; k < 8; k += 2) {
+            const float p0 = rv ? ex2_approx(s[c + k] - m[c + k]) : 0.f;
+            const float p1 = rv ? ex2_approx(s[c + k + 1] - m[c + k + 1]) : 0.f;
+            lsum[c + k] += p0;
+            lsum[c + k + 1] += p1;
+            w[k >> 1] = pack_bf16x2(p0, p1);
+          }
+          const int chunk = ((h0 + c) >> 3) ^ sw;
+          *reinterpret_cast<uint4*>(pb + chunk * 16) = make_uint4(w[0], w[1], w[2], w[3]);
         }
         if (!rv) {
           // rows past the sequence end may hold anything: zero them so 0 * garbage cannot reach O
