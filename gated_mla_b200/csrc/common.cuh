@@ -105,7 +105,7 @@ static __device__ __noinline__ float rope_rotate(float v, float partner, bool od
 }
 
 __device__ __forceinline__ void epi_store(const EpiSeg& e, int64_t row, int f, float v, int t = 0) {
-  if (e.gate) v *= 1.f / (1.f + __expf(-e.gate[static_cast<int64_t>(t) * e.gate_stride + f / e.gate_div]));
+  if (e.gate) v *= __fdividef(1.f, 1.f + __expf(-e.gate[static_cast<int64_t>(t) * e.gate_stride + f / e.gate_div]));
   const int64_t off = row * e.row_stride + static_cast<int64_t>(f / e.block) * e.block_stride + (f % e.block) +
                       e.col_offset;
   if (e.bias) v += e.bias[f];

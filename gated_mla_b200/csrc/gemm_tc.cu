@@ -146,6 +146,7 @@ __global__ void __launch_bounds__(192, 1) gemm_bf16_tc_kernel(const __grid_const
   if (threadIdx.x == 0) griddep_launch_dependents();
   const uint32_t tmem = *tmem_slot;
 
+  float gl0[16];   // epilogue warps, swap orientation: see below
   if (warp == 0) {
     if (lane == 0) {
       const CUtensorMap* wmap = &a.wt[tile.seg];
@@ -222,33 +223,50 @@ __global__ void __launch_bounds__(192, 1) gemm_bf16_tc_kernel(const __grid_const
     const int q = warp & 3;
     const int r = q * 32 + lane;            // accumulator row of this thread
     griddep_wait();                         // before reading positions or writing outputs
+    // by value: a runtime-indexed reference into the parameter space costs a
+    // chain of constant-bank loads on every use
+    const EpiSeg e = a.epi[tile.seg];
+    const int seg_rows = a.seg_rows[tile.seg];
+    if (kSwap) {
+      // While the MMAs run: the tile's token -> output row / position table (built
+      // once in shared memory so the store loop has no dependent global loads), and
+      // the gate-logit lines this warp will read brought into L1.
+      for (int lt = threadIdx.x - 64; lt < BN; lt += 128) {
+        const int tok = tile.tok0 + lt;
+        int64_t row = tok;
+        int pos = 0;
+        if (lt < tile.ntok && (e.rope || e.cache_scatter)) pos = a.positions[tok];
+        if (lt < tile.ntok && e.cache_scatter) {
+          row = cache_row(a.cache, a.seq_ids[tok], pos);
+          if (row < 0) report_status(a.status, kStatusRange);
+        }
+        tok_row[lt] = lt < tile.ntok ? row : -1;
+        tok_pos[lt] = pos;
+      }
+      asm volatile("bar.sync 2, 128;" ::: "memory");
+    }
+    // the gate logits of the first 16 tokens this thread stores (all of them in the
+    // few-token case), loaded before the accumulator is ready
+    {
+      const int f = tile.wrow0 + r;
+      const int c_lo = split ? static_cast<int>(rank) * cpr : 0;
+      const int c_hi = split ? c_lo + own_cols : BN;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int lt = c_lo + j;
+        gl0[j] = (kSwap && e.gate && f < seg_rows && lt < c_hi && lt < tile.ntok)
+                     ? e.gate[static_cast<int64_t>(tile.tok0 + lt) * e.gate_stride + f / e.gate_div]
+                     : 0.f;
+      }
+    }
     // Split-K epilogues meet at named barrier 2; a failed wait still walks the
     // same barriers (with its stores skipped) so the four warps stay in step.
     const bool acc_ok = mbar_wait(acc_full, 0, abort_flag, a.status);
     if (acc_ok || kSwap) {
       tc_fence_after();
-      // by value: a runtime-indexed reference into the parameter space costs a
-      // chain of constant-bank loads on every use
-      const EpiSeg e = a.epi[tile.seg];
-      const int seg_rows = a.seg_rows[tile.seg];
       if (kSwap) {
-        // row r = weight feature, columns = tokens. The tile's token -> output
-        // row / position table is built once in shared memory so the store loop
-        // has no dependent global loads.
+        // row r = weight feature, columns = tokens
         const int f = tile.wrow0 + r;
-        for (int lt = threadIdx.x - 64; lt < BN; lt += 128) {
-          const int tok = tile.tok0 + lt;
-          int64_t row = tok;
-          int pos = 0;
-          if (lt < tile.ntok && (e.rope || e.cache_scatter)) pos = a.positions[tok];
-          if (lt < tile.ntok && e.cache_scatter) {
-            row = cache_row(a.cache, a.seq_ids[tok], pos);
-            if (row < 0) report_status(a.status, kStatusRange);
-          }
-          tok_row[lt] = lt < tile.ntok ? row : -1;
-          tok_pos[lt] = pos;
-        }
-        asm volatile("bar.sync 2, 128;" ::: "memory");
         // this thread's feature is fixed: hoist its column offset, bias and gate index
         const int64_t colpart =
             static_cast<int64_t>(f / e.block) * e.block_stride + (f % e.block) + e.col_offset;
@@ -262,9 +280,10 @@ __global__ void __launch_bounds__(192, 1) gemm_bf16_tc_kernel(const __grid_const
           if (e.gate) {
 #pragma unroll
             for (int j = 0; j < 16; ++j)
-              gl[j] = (tok_row[c0 + j] >= 0 && f_ok)
-                          ? e.gate[static_cast<int64_t>(tile.tok0 + c0 + j) * e.gate_stride + gcol]
-                          : 0.f;
+              gl[j] = c0 == 0 ? gl0[j]
+                              : ((tok_row[c0 + j] >= 0 && f_ok)
+                                     ? e.gate[static_cast<int64_t>(tile.tok0 + c0 + j) * e.gate_stride + gcol]
+                                     : 0.f);
           }
 #pragma unroll 4
           for (int j = 0; j < 16; ++j) {
@@ -278,7 +297,7 @@ __global__ void __launch_bounds__(192, 1) gemm_bf16_tc_kernel(const __grid_const
             const int64_t row = tok_row[tl];
             if (row < 0 || !f_ok) continue;
             val += fbias;
-            if (e.gate) val *= 1.f / (1.f + __expf(-gl[j]));
+            if (e.gate) val *= __fdividef(1.f, 1.f + __expf(-gl[j]));
             const int64_t off = row * e.row_stride + colpart;
             if (e.out_f32)
               static_cast<float*>(e.out)[off] = val;
@@ -421,9 +440,10 @@ __global__ void __launch_bounds__(192, 1) gemm_bf16_tc_kernel(const __grid_const
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
               const int tl = col0 + c + j;
-              gl[j] = (j < nc && tok_row[tl] >= 0 && f_ok)
-                          ? e.gate[static_cast<int64_t>(tile.tok0 + tl) * e.gate_stride + gcol]
-                          : 0.f;
+              gl[j] = c == 0 ? gl0[j]
+                             : ((j < nc && tok_row[tl] >= 0 && f_ok)
+                                    ? e.gate[static_cast<int64_t>(tile.tok0 + tl) * e.gate_stride + gcol]
+                                    : 0.f);
             }
           }
           float x[16];
@@ -455,7 +475,7 @@ __global__ void __launch_bounds__(192, 1) gemm_bf16_tc_kernel(const __grid_const
             const int64_t row = tok_row[tl];
             if (row < 0 || !f_ok || !got) continue;
             val += fbias;
-            if (e.gate) val *= 1.f / (1.f + __expf(-gl[j]));
+            if (e.gate) val *= __fdividef(1.f, 1.f + __expf(-gl[j]));
             const int64_t off = row * e.row_stride + colpart;
             if (e.out_f32)
               static_cast<float*>(e.out)[off] = val;

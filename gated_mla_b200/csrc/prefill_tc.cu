@@ -305,7 +305,7 @@ __global__ void __launch_bounds__(576, 1) prefill_attn_kernel(const __grid_const
       const int64_t tok = beg + qi;
       const float inv = 1.f / l;
       float gh = 1.f;
-      if (valid && a.gate_logits && a.gate_mode != 0) gh = 1.f / (1.f + __expf(-__ldg(a.gate_logits + tok * G + h)));
+      if (valid && a.gate_logits && a.gate_mode != 0) gh = __fdividef(1.f, 1.f + __expf(-__ldg(a.gate_logits + tok * G + h)));
 #pragma unroll 1
       for (int c = c0; c < c0 + 64; c += 32) {
         uint32_t w[32];
@@ -322,7 +322,7 @@ __global__ void __launch_bounds__(576, 1) prefill_attn_kernel(const __grid_const
           float o[8];
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
-            const float gk = a.gate_mode == 0 && a.gate_logits ? 1.f / (1.f + __expf(-g[i + k])) : gh;
+            const float gk = a.gate_mode == 0 && a.gate_logits ? __fdividef(1.f, 1.f + __expf(-g[i + k])) : gh;
             o[k] = __uint_as_float(w[i + k]) * inv * gk;
           }
           uint4 pk;
