@@ -496,22 +496,25 @@ __global__ void __launch_bounds__(64 + 128 * (HG >= 32 ? 2 : 1), 1) decode_attn_
         const bool first = (t == sg.y);
         ok = ok && mbar_wait(&sm->s_full, ntile & 1, abort_flag, a.status);
         tc_fence_after();
-        float s[HT];
-#pragma unroll
-        for (int c = 0; c < HT; c += 16) {
-          uint32_t v[16];
-          tmem_ld16(tmem + (ntile & 1) * HG + lane_off + h0 + c, v);
-          tmem_ld_wait();
-#pragma unroll
-          for (int j = 0; j < 16; ++j) s[c + j] = __uint_as_float(v[j]);
-        }
+        // Scores are read from TMEM 16 heads at a time, once for the max test and
+        // again for P, so no thread holds all its heads' scores at once.
+        const uint32_t tS = tmem + (ntile & 1) * HG + lane_off + h0;
         const int valid = min(kTileTok, L - t * kTileTok);
         const bool rv = row < valid;
+        auto load16 = [&](int c, float (&x)[16]) {
+          uint32_t v[16];
+          tmem_ld16(tS + c, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) x[j] = rv ? __uint_as_float(v[j]) : NEG_INF;
+        };
         bool need = first;
 #pragma unroll
-        for (int h = 0; h < HT; ++h) {
-          if (!rv) s[h] = NEG_INF;
-          need |= s[h] > m[h] + 8.f;
+        for (int c = 0; c < HT; c += 16) {
+          float x[16];
+          load16(c, x);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) need |= x[j] > m[c + j] + 8.f;
         }
         // block-wide vote among the softmax threads
         const int par = ntile & 1;
@@ -521,42 +524,48 @@ __global__ void __launch_bounds__(64 + 128 * (HG >= 32 ? 2 : 1), 1) decode_attn_
         if (ltid == 0) sm->vote[par ^ 1] = 0;
         if (need_all) {
 #pragma unroll
-          for (int h = 0; h < HT; ++h) {
-            const int k = __reduce_max_sync(0xffffffffu, float_to_ordered(s[h]));
-            if (lane == 0) sm->red[par][q4][h0 + h] = k;
+          for (int c = 0; c < HT; c += 16) {
+            float x[16];
+            load16(c, x);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const int k = __reduce_max_sync(0xffffffffu, float_to_ordered(x[j]));
+              if (lane == 0) sm->red[par][q4][h0 + c + j] = k;
+            }
           }
           asm volatile("bar.sync 1, %0;" ::"n"(128 * SG) : "memory");
-          float alpha[HT];
-          bool rescale = false;
 #pragma unroll
-          for (int h = 0; h < HT; ++h) {
-            int k = sm->red[par][0][h0 + h];
-            k = max(k, sm->red[par][1][h0 + h]);
-            k = max(k, sm->red[par][2][h0 + h]);
-            k = max(k, sm->red[par][3][h0 + h]);
-            const float tmax = ordered_to_float(k);
-            const float mn = fmaxf(m[h], tmax);
-            alpha[h] = (m[h] == NEG_INF) ? 0.f : ex2_approx(m[h] - mn);
-            rescale |= (mn > m[h]) && !first;
-            m[h] = mn;
-            lsum[h] *= alpha[h];
-          }
-          if (rescale) {
-            // O^T columns of head h scale by alpha[h] (O of the previous tile is complete:
-            // S of this tile was committed after it)
+          for (int c = 0; c < HT; c += 16) {
+            float alpha[16];
+            bool rescale = false;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const int h = c + j;
+              int k = sm->red[par][0][h0 + h];
+              k = max(k, sm->red[par][1][h0 + h]);
+              k = max(k, sm->red[par][2][h0 + h]);
+              k = max(k, sm->red[par][3][h0 + h]);
+              const float tmax = ordered_to_float(k);
+              const float mn = fmaxf(m[h], tmax);
+              alpha[j] = (m[h] == NEG_INF) ? 0.f : ex2_approx(m[h] - mn);
+              rescale |= (mn > m[h]) && !first;
+              m[h] = mn;
+              lsum[h] *= alpha[j];
+            }
+            if (rescale) {
+              // O^T columns of these heads scale by alpha (O of the previous tile is
+              // complete: S of this tile was committed after it)
 #pragma unroll 1
-            for (int mc = 0; mc < kNcBox / 2; ++mc) {
-#pragma unroll
-              for (int c = 0; c < HT; c += 16) {
+              for (int mc = 0; mc < kNcBox / 2; ++mc) {
                 uint32_t v[16];
                 tmem_ld16(tO + lane_off + mc * HG + h0 + c, v);
                 tmem_ld_wait();
 #pragma unroll
-                for (int j = 0; j < 16; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * alpha[c + j]);
+                for (int j = 0; j < 16; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * alpha[j]);
                 tmem_st16(tO + lane_off + mc * HG + h0 + c, v);
               }
+              tmem_st_wait();
             }
-            tmem_st_wait();
           }
         }
         // P = exp2(s - m) as bf16, this thread's token row of P[token][head]: 16-byte
@@ -564,18 +573,24 @@ __global__ void __launch_bounds__(64 + 128 * (HG >= 32 ? 2 : 1), 1) decode_attn_
         uint8_t* pb = pbuf + row * (HG * 2);
         const int sw = HG == 64 ? (row & 7) : (HG == 32 ? ((row >> 1) & 3) : ((row >> 2) & 1));
 #pragma unroll
-        for (int c = 0; c < HT; c += 8) {
-          uint32_t w[4];
+        for (int c = 0; c < HT; c += 16) {
+          float x[16];
+          load16(c, x);
 #pragma unroll
-          for (int k = 0; k < 8; k += 2) {
-            const float p0 = rv ? ex2_approx(s[c + k] - m[c + k]) : 0.f;
-            const float p1 = rv ? ex2_approx(s[c + k + 1] - m[c + k + 1]) : 0.f;
-            lsum[c + k] += p0;
-            lsum[c + k + 1] += p1;
-            w[k >> 1] = pack_bf16x2(p0, p1);
+          for (int c8 = 0; c8 < 16; c8 += 8) {
+            uint32_t w[4];
+#pragma unroll
+            for (int k = 0; k < 8; k += 2) {
+              const int h = c + c8 + k;
+              const float p0 = rv ? ex2_approx(x[c8 + k] - m[h]) : 0.f;
+              const float p1 = rv ? ex2_approx(x[c8 + k + 1] - m[h + 1]) : 0.f;
+              lsum[h] += p0;
+              lsum[h + 1] += p1;
+              w[k >> 1] = pack_bf16x2(p0, p1);
+            }
+            const int chunk = ((h0 + c + c8) >> 3) ^ sw;
+            *reinterpret_cast<uint4*>(pb + chunk * 16) = make_uint4(w[0], w[1], w[2], w[3]);
           }
-          const int chunk = ((h0 + c) >> 3) ^ sw;
-          *reinterpret_cast<uint4*>(pb + chunk * 16) = make_uint4(w[0], w[1], w[2], w[3]);
         }
         if (!rv) {
           // rows past the sequence end may hold anything: zero them so 0 * garbage cannot reach O
