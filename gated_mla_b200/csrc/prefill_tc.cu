@@ -12,8 +12,8 @@
 // columns); the softmax writes P (bf16) over the first half of S's columns
 // and the P V product reads it from there as the A operand, so P never goes
 // through shared memory.
-// Roles: warp 0 TMA, one thread of warp 1 the MMAs, warps 2..9 the softmax
-// and epilogue of tile A (half a query row per thread), warps 10..17 those of B.
+// Roles: warp 0 TMA, one thread of warp 1 the MMAs, warps 2..5 the softmax
+// and epilogue of tile A (one query row per thread), warps 6..9 those of B.
 // The running max of a row is raised only when a tile's max exceeds it by
 // more than 2^8 (the final normalisation uses the same reference, so the
 // result is exact); O is rescaled in TMEM only then.
@@ -30,7 +30,7 @@ constexpr int kD = 128;           // head dim
 constexpr int kBox = 128 * 128;   // one [128 rows x 64] bf16 box: 16 KB
 constexpr int kTile = 2 * kBox;   // [128 rows x 128] bf16
 constexpr int kStages = 2;
-constexpr int kSmem = 2 * kTile + kStages * 2 * kTile + 1024 + 2304;
+constexpr int kSmem = 2 * kTile + kStages * 2 * kTile + 1024 + 256;
 constexpr uint32_t kTmemCols = 512;   // per tile: S/P 128 columns + O 128 columns
 
 struct PfBars {
@@ -40,11 +40,10 @@ struct PfBars {
   uint64_t drain;
   uint32_t tmem;
   int abort;
-  float xmax[2][2 * 128];   // per tile: the two halves' partial row maxima (then row sums)
 };
 }  // namespace
 
-__global__ void __launch_bounds__(576, 1) prefill_attn_kernel(const __grid_constant__ PrefillArgs a) {
+__global__ void __launch_bounds__(320, 1) prefill_attn_kernel(const __grid_constant__ PrefillArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;                             // [tile A, tile B]
@@ -74,7 +73,7 @@ __global__ void __launch_bounds__(576, 1) prefill_attn_kernel(const __grid_const
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars->s_full[i], 1);
-      mbar_init(&bars->p_full[i], 256);
+      mbar_init(&bars->p_full[i], 128);
       mbar_init(&bars->o_done[i], 1);
     }
     mbar_init(&bars->drain, 1);
@@ -191,111 +190,133 @@ __global__ void __launch_bounds__(576, 1) prefill_attn_kernel(const __grid_const
     }
   } else {
     // ------------------------- softmax + epilogue of one tile -------------------------
-    // Eight warps per tile: warps of the same TMEM lane quarter split a query
-    // row into two halves of 64 keys (and 64 output columns). The halves swap
-    // their partial row maxima through shared memory at a named barrier (one
-    // per tile); each keeps its own partial row sum until the end.
-    const int x = warp < 10 ? 0 : 1;
-    const int gw = warp - (x == 0 ? 2 : 10);      // 0..7 within the tile's group
-    const int half = gw >> 2;
+    // Four warps per tile, one query row per thread: 128 keys per tile step and
+    // 128 output columns at the end.
+    const int x = warp < 6 ? 0 : 1;
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;                 // query row in the tile
     const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
     const uint32_t tS = tmem + 256 * x + lane_off, tO = tS + 128;
-    const int c0 = half * 64;                     // this thread's key / output columns
     const int qt = x == 0 ? qtA : qtB;
     const int qi = qt * kBQ + r;                  // position in the sequence
     const float NEG_INF = -__int_as_float(0x7f800000);
-    float* xmax = bars->xmax[x];                  // [2 halves][128 rows]
     float m = NEG_INF, l = 0.f;
     bool ok = true;
     const bool active = x == 0 || hasB;
-    const uint32_t bar_id = 1 + x;
+    const uint64_t sc2 = f2_pack(a.scale_log2, a.scale_log2);
+    // P = exp2(s*scale - m) for 32 keys [k0, k0 + 32) as 16 bf16 pairs, stored
+    // over S at columns [k0/2, k0/2 + 16); returns the sum of the 32 values
+    auto p_chunk = [&](const uint32_t (&u)[32], int k0, bool diag, uint64_t nm2) -> uint64_t {
+      uint32_t pk[16];
+      uint64_t ls2[2] = {0ull, 0ull};
+#pragma unroll
+      for (int i = 0; i < 32; i += 2) {
+        float x0, x1, p0, p1;
+        f2_unpack(ffma2(f2_pack(__uint_as_float(u[i]), __uint_as_float(u[i + 1])), sc2, nm2), x0, x1);
+        if ((i & 2) == 0) {   // half the exponentials on the special-function unit,
+          p0 = ex2_approx(x0);
+          p1 = ex2_approx(x1);
+        } else {              // half on the FMA pipes
+          exp2_poly2(x0, x1, p0, p1);
+        }
+        if (diag) {
+          p0 = (k0 + i <= r) ? p0 : 0.f;
+          p1 = (k0 + i + 1 <= r) ? p1 : 0.f;
+        }
+        ls2[(i >> 1) & 1] = fadd2(ls2[(i >> 1) & 1], f2_pack(p0, p1));
+        pk[i >> 1] = pack_bf16x2(p0, p1);
+      }
+      tmem_st16(tS + (k0 >> 1), pk);
+      return fadd2(ls2[0], ls2[1]);
+    };
     for (int j = 0; active && j <= qt; ++j) {
       ok = ok && mbar_wait(&bars->s_full[x], j & 1, abort_flag, a.status);
       tc_fence_after();
       const bool diag = (j == qt);
-      uint32_t v[64];
-      tmem_ld32(tS + c0, *reinterpret_cast<uint32_t(*)[32]>(v));
-      tmem_ld32(tS + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
-      tmem_ld_wait();
-      // partial row max of the raw scores (the scale is positive)
+      // the row max of the raw scores (the scale is positive); keys 64..127 stay
+      // in registers, keys 0..63 are read again for P
+      uint32_t v0[32], v1[32];
       float pm[4];
 #pragma unroll
       for (int k = 0; k < 4; ++k) pm[k] = NEG_INF;
+      {
+        uint32_t u0[32], u1[32];
+        tmem_ld32(tS, u0);
+        tmem_ld32(tS + 32, u1);
+        tmem_ld_wait();
+        if (!diag) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            pm[0] = fmax3(pm[0], __uint_as_float(u0[i]), __uint_as_float(u0[i + 1]));
+            pm[1] = fmax3(pm[1], __uint_as_float(u1[i]), __uint_as_float(u1[i + 1]));
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            if (i <= r) pm[0] = fmaxf(pm[0], __uint_as_float(u0[i]));
+            if (32 + i <= r) pm[1] = fmaxf(pm[1], __uint_as_float(u1[i]));
+          }
+        }
+      }
+      tmem_ld32(tS + 64, v0);
+      tmem_ld32(tS + 96, v1);
+      tmem_ld_wait();
       if (!diag) {
 #pragma unroll
-        for (int i = 0; i < 64; i += 2)
-          pm[(i >> 1) & 3] = fmax3(pm[(i >> 1) & 3], __uint_as_float(v[i]), __uint_as_float(v[i + 1]));
+        for (int i = 0; i < 32; i += 2) {
+          pm[2] = fmax3(pm[2], __uint_as_float(v0[i]), __uint_as_float(v0[i + 1]));
+          pm[3] = fmax3(pm[3], __uint_as_float(v1[i]), __uint_as_float(v1[i + 1]));
+        }
       } else {
 #pragma unroll
-        for (int i = 0; i < 64; ++i)
-          if (c0 + i <= r) pm[i & 3] = fmaxf(pm[i & 3], __uint_as_float(v[i]));
+        for (int i = 0; i < 32; ++i) {
+          if (64 + i <= r) pm[2] = fmaxf(pm[2], __uint_as_float(v0[i]));
+          if (96 + i <= r) pm[3] = fmaxf(pm[3], __uint_as_float(v1[i]));
+        }
       }
-      xmax[half * 128 + r] = fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3]));
-      // both halves' S loads are complete here, so P may overwrite S after it
-      asm volatile("bar.sync %0, 256;" ::"r"(bar_id) : "memory");
-      const float tmax = fmaxf(xmax[r], xmax[128 + r]) * a.scale_log2;
+      const float tmax = fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])) * a.scale_log2;
       if (j == 0 || tmax > m + 8.f) {
         const float mn = fmaxf(m, tmax);
         const float alpha = (m == NEG_INF) ? 0.f : ex2_approx(m - mn);
         if (j > 0 && alpha != 1.f) {
           // O of the previous tile is complete: S of this tile was issued after it
 #pragma unroll 1
-          for (int c = 0; c < 64; c += 16) {
+          for (int c = 0; c < 128; c += 16) {
             uint32_t w[16];
-            tmem_ld16(tO + c0 + c, w);
+            tmem_ld16(tO + c, w);
             tmem_ld_wait();
 #pragma unroll
             for (int k = 0; k < 16; ++k) w[k] = __float_as_uint(__uint_as_float(w[k]) * alpha);
-            tmem_st16(tO + c0 + c, w);
+            tmem_st16(tO + c, w);
           }
           tmem_st_wait();
         }
         l *= alpha;
         m = mn;
       }
-      // P = exp2(s*scale - m) as bf16 pairs: keys [c0, c0 + 64) -> columns [c0/2, c0/2 + 32)
-      const uint64_t sc2 = f2_pack(a.scale_log2, a.scale_log2), nm2 = f2_pack(-m, -m);
-      uint64_t ls2[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) ls2[k] = 0ull;
-#pragma unroll
-      for (int c = 0; c < 64; c += 32) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          float x0, x1, p0, p1;
-          f2_unpack(ffma2(f2_pack(__uint_as_float(v[c + i]), __uint_as_float(v[c + i + 1])), sc2, nm2), x0, x1);
-          if ((i & 2) == 0) {   // half the exponentials on the special-function unit,
-            p0 = ex2_approx(x0);
-            p1 = ex2_approx(x1);
-          } else {              // half on the FMA pipes
-            exp2_poly2(x0, x1, p0, p1);
-          }
-          if (diag) {
-            p0 = (c0 + c + i <= r) ? p0 : 0.f;
-            p1 = (c0 + c + i + 1 <= r) ? p1 : 0.f;
-          }
-          ls2[(i >> 1) & 3] = fadd2(ls2[(i >> 1) & 3], f2_pack(p0, p1));
-          pk[i >> 1] = pack_bf16x2(p0, p1);
-        }
-        tmem_st16(tS + ((c0 + c) >> 1), pk);
+      // P over S: keys [0, 64) are read again (P of a 32-key chunk only overwrites
+      // columns whose scores this thread has already read)
+      const uint64_t nm2 = f2_pack(-m, -m);
+      uint64_t ls = 0ull;
+      {
+        uint32_t u[32];
+        tmem_ld32(tS, u);
+        tmem_ld_wait();
+        ls = fadd2(ls, p_chunk(u, 0, diag, nm2));
+        tmem_ld32(tS + 32, u);
+        tmem_ld_wait();
+        ls = fadd2(ls, p_chunk(u, 32, diag, nm2));
       }
+      ls = fadd2(ls, p_chunk(v0, 64, diag, nm2));
+      ls = fadd2(ls, p_chunk(v1, 96, diag, nm2));
       {
         float s0, s1;
-        f2_unpack(fadd2(fadd2(ls2[0], ls2[1]), fadd2(ls2[2], ls2[3])), s0, s1);
+        f2_unpack(ls, s0, s1);
         l += s0 + s1;
       }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&bars->p_full[x]);
-    }
-    // row sum of both halves
-    if (active) {
-      xmax[half * 128 + r] = l;
-      asm volatile("bar.sync %0, 256;" ::"r"(bar_id) : "memory");
-      l = xmax[r] + xmax[128 + r];
     }
     if (active && ok && mbar_wait(&bars->o_done[x], 0, abort_flag, a.status)) {
       tc_fence_after();
@@ -307,7 +328,7 @@ __global__ void __launch_bounds__(576, 1) prefill_attn_kernel(const __grid_const
       float gh = 1.f;
       if (valid && a.gate_logits && a.gate_mode != 0) gh = __fdividef(1.f, 1.f + __expf(-__ldg(a.gate_logits + tok * G + h)));
 #pragma unroll 1
-      for (int c = c0; c < c0 + 64; c += 32) {
+      for (int c = 0; c < 128; c += 32) {
         uint32_t w[32];
         tmem_ld32(tO + c, w);
         tmem_ld_wait();
@@ -350,7 +371,7 @@ cudaError_t launch_prefill_attn_bf16(const PrefillArgs& a, cudaStream_t st) {
   if (e != cudaSuccess) return e;
   const int pairs = (a.q_tiles_per_seq + 1) / 2;
   prof_begin(st, "prefill_attn");
-  e = launch_pdl(prefill_attn_kernel, dim3(pairs, a.H, a.B), dim3(576), kSmem, st, 1, a);
+  e = launch_pdl(prefill_attn_kernel, dim3(pairs, a.H, a.B), dim3(320), kSmem, st, 1, a);
   prof_end(st);
   return e;
 }
