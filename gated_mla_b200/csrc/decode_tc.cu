@@ -651,6 +651,9 @@ __global__ void __launch_bounds__(64 + 128 * (HG >= 32 ? 2 : 1), 1) decode_attn_
     }
   }
 
+  // one lane of a warp ran a role alone: reconverge before the block-wide barrier
+  // (a partly arrived warp must not count as arrived)
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

@@ -487,6 +487,9 @@ __global__ void __launch_bounds__(192, 1) gemm_bf16_tc_kernel(const __grid_const
     }
   }
 
+  // one lane of a warp ran a role alone: reconverge before the block-wide barrier
+  // (a partly arrived warp must not count as arrived)
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

@@ -156,6 +156,7 @@ __global__ void __launch_bounds__(320, 1) prefill_attn_kernel(const __grid_const
           if (!mbar_wait(&bars->p_full[0], j & 1, abort_flag, a.status)) { ok = false; break; }
           tc_fence_after();
           issue_o(0, j);
+          if (j == qtA) umma_commit(&bars->o_done[0]);   // tile A's epilogue overlaps B's last step
           if (j + 1 <= qtA) {
             if (!mbar_wait(&bars->kv_full[(j + 1) % kStages], ((j + 1) / kStages) & 1, abort_flag, a.status)) {
               ok = false;
@@ -181,7 +182,6 @@ __global__ void __launch_bounds__(320, 1) prefill_attn_kernel(const __grid_const
         }
       }
       if (ok) {
-        umma_commit(&bars->o_done[0]);
         umma_commit(&bars->o_done[1]);
       } else {
         umma_commit(&bars->drain);
@@ -230,6 +230,13 @@ __global__ void __launch_bounds__(320, 1) prefill_attn_kernel(const __grid_const
       return fadd2(ls2[0], ls2[1]);
     };
     for (int j = 0; active && j <= qt; ++j) {
+      if (j == max(0, qt - 2) && a.gate_logits && qi < len) {
+        // this row's gate logits, needed by the epilogue, requested into L2 now
+        const int G = a.gate_mode == 0 ? a.H * kD : a.H;
+        const float* gr = a.gate_logits + static_cast<int64_t>(beg + qi) * G + (a.gate_mode == 0 ? h * kD : h);
+#pragma unroll
+        for (int c = 0; c < (a.gate_mode == 0 ? 4 : 1); ++c) prefetch_l2(gr + c * 32);
+      }
       ok = ok && mbar_wait(&bars->s_full[x], j & 1, abort_flag, a.status);
       tc_fence_after();
       const bool diag = (j == qt);
@@ -334,9 +341,17 @@ __global__ void __launch_bounds__(320, 1) prefill_attn_kernel(const __grid_const
         tmem_ld_wait();
         if (!valid) continue;
         float g[32];
+        if (a.gate_logits && a.gate_mode == 0) {
+          const float4* gp = reinterpret_cast<const float4*>(a.gate_logits + tok * G + h * kD + c);
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
-          g[i] = (a.gate_logits && a.gate_mode == 0) ? __ldg(a.gate_logits + tok * G + h * kD + c + i) : 0.f;
+          for (int i = 0; i < 8; ++i) {
+            const float4 q4v = __ldg(gp + i);
+            g[4 * i] = q4v.x;
+            g[4 * i + 1] = q4v.y;
+            g[4 * i + 2] = q4v.z;
+            g[4 * i + 3] = q4v.w;
+          }
+        }
         uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) + tok * HD + h * kD + c);
 #pragma unroll
         for (int i = 0; i < 32; i += 8) {
@@ -357,6 +372,9 @@ __global__ void __launch_bounds__(320, 1) prefill_attn_kernel(const __grid_const
     }
   }
 
+  // one lane of a warp ran a role alone: reconverge before the block-wide barrier
+  // (a partly arrived warp must not count as arrived)
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
