@@ -230,7 +230,7 @@ __global__ void __launch_bounds__(320, 1) prefill_attn_kernel(const __grid_const
       return fadd2(ls2[0], ls2[1]);
     };
     for (int j = 0; active && j <= qt; ++j) {
-      if (j == max(0, qt - 2) && a.gate_logits && qi < len) {
+      if (j == max(0, qt - 4) && a.gate_logits && qi < len) {
         // this row's gate logits, needed by the epilogue, requested into L2 now
         const int G = a.gate_mode == 0 ? a.H * kD : a.H;
         const float* gr = a.gate_logits + static_cast<int64_t>(beg + qi) * G + (a.gate_mode == 0 ? h * kD : h);
@@ -336,12 +336,9 @@ __global__ void __launch_bounds__(320, 1) prefill_attn_kernel(const __grid_const
       if (valid && a.gate_logits && a.gate_mode != 0) gh = __fdividef(1.f, 1.f + __expf(-__ldg(a.gate_logits + tok * G + h)));
 #pragma unroll 1
       for (int c = 0; c < 128; c += 32) {
-        uint32_t w[32];
-        tmem_ld32(tO + c, w);
-        tmem_ld_wait();
-        if (!valid) continue;
+        // the gate logits first, so their latency overlaps the TMEM read
         float g[32];
-        if (a.gate_logits && a.gate_mode == 0) {
+        if (valid && a.gate_logits && a.gate_mode == 0) {
           const float4* gp = reinterpret_cast<const float4*>(a.gate_logits + tok * G + h * kD + c);
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
@@ -352,13 +349,17 @@ __global__ void __launch_bounds__(320, 1) prefill_attn_kernel(const __grid_const
             g[4 * i + 3] = q4v.w;
           }
         }
+        uint32_t w[32];
+        tmem_ld32(tO + c, w);
+        tmem_ld_wait();
+        if (!valid) continue;
         uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) + tok * HD + h * kD + c);
 #pragma unroll
         for (int i = 0; i < 32; i += 8) {
           float o[8];
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
-            const float gk = a.gate_mode == 0 && a.gate_logits ? __fdividef(1.f, 1.f + __expf(-g[i + k])) : gh;
+            const float gk = a.gate_mode == 0 && a.gate_logits ? sigmoid_tanh(g[i + k]) : gh;
             o[k] = __uint_as_float(w[i + k]) * inv * gk;
           }
           uint4 pk;
