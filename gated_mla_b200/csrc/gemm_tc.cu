@@ -21,18 +21,21 @@
 
 namespace gmla {
 
-template <int BN>
+template <int BN, bool kSwap>
 struct GemmCfg {
   static constexpr int kABytes = 128 * 128;              // 128 rows x 64 bf16
   static constexpr int kBBytes = BN * 128;               // BN rows x 64 bf16
   static constexpr int kStageBytes = kABytes + kBBytes;
-  // narrow tiles (few tokens, weight streaming): 4 stages so two CTAs share an SM
-  static constexpr int kStages = (BN >= 256) ? 4 : (BN >= 128 ? 6 : 4);
+  // Few tokens (weight streaming): 4 stages, narrow tiles let two CTAs share an SM.
+  // Many tokens: two CTAs per SM with 96 KB of stages each, so one CTA's epilogue
+  // runs while the other's MMAs keep the tensor pipe busy.
+  static constexpr int kStages = kSwap ? ((BN >= 256) ? 4 : (BN >= 128 ? 6 : 4)) : (BN >= 256 ? 2 : 3);
+  static constexpr int kCtasPerSm = kSwap ? 1 : 2;
   static constexpr int kTmemCols = BN < 32 ? 32 : BN;
   static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/ + 12 * BN;
   // split-K partials are received into the (then idle) stage memory:
   // splits x 128 x cpr fp32 with splits <= 8 and cpr = ceil4(ceil(BN / splits)) <= BN / splits + 3
-  static_assert(128 * 4 * (BN + 24) <= kStages * kStageBytes, "split-K receive buffer");
+  static_assert(!kSwap || 128 * 4 * (BN + 24) <= kStages * kStageBytes, "split-K receive buffer");
 };
 
 struct GemmTile {
@@ -89,8 +92,8 @@ __device__ __forceinline__ bool gemm_tile(const GemmArgs& a, GemmTile& t) {
 }
 
 template <int BN, bool kSwap>
-__global__ void __launch_bounds__(192, 1) gemm_bf16_tc_kernel(const __grid_constant__ GemmArgs a) {
-  using C = GemmCfg<BN>;
+__global__ void __launch_bounds__(192, kSwap ? 1 : 2) gemm_bf16_tc_kernel(const __grid_constant__ GemmArgs a) {
+  using C = GemmCfg<BN, kSwap>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
@@ -500,7 +503,7 @@ __global__ void __launch_bounds__(192, 1) gemm_bf16_tc_kernel(const __grid_const
 
 template <int BN, bool kSwap>
 static cudaError_t launch_one(const GemmArgs& a, dim3 grid, cudaStream_t st, const char* name) {
-  using C = GemmCfg<BN>;
+  using C = GemmCfg<BN, kSwap>;
   auto k = gemm_bf16_tc_kernel<BN, kSwap>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
