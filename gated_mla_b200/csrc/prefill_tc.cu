@@ -240,45 +240,46 @@ __global__ void __launch_bounds__(320, 1) prefill_attn_kernel(const __grid_const
       ok = ok && mbar_wait(&bars->s_full[x], j & 1, abort_flag, a.status);
       tc_fence_after();
       const bool diag = (j == qt);
-      // the row max of the raw scores (the scale is positive); keys 64..127 stay
-      // in registers, keys 0..63 are read again for P
-      uint32_t v0[32], v1[32];
+      // the row max of the raw scores (the scale is positive): keys 64..127 are
+      // read while keys 0..63 are scanned
       float pm[4];
 #pragma unroll
       for (int k = 0; k < 4; ++k) pm[k] = NEG_INF;
       {
-        uint32_t u0[32], u1[32];
-        tmem_ld32(tS, u0);
-        tmem_ld32(tS + 32, u1);
-        tmem_ld_wait();
+        uint32_t c0[32], c1[32], c2[32], c3[32];
+        tmem_ld32(tS, c0);
+        tmem_ld32(tS + 32, c1);
+        tmem_ld_wait_regs(c0);
+        tmem_ld_wait_regs(c1);
+        tmem_ld32(tS + 64, c2);
+        tmem_ld32(tS + 96, c3);
         if (!diag) {
 #pragma unroll
           for (int i = 0; i < 32; i += 2) {
-            pm[0] = fmax3(pm[0], __uint_as_float(u0[i]), __uint_as_float(u0[i + 1]));
-            pm[1] = fmax3(pm[1], __uint_as_float(u1[i]), __uint_as_float(u1[i + 1]));
+            pm[0] = fmax3(pm[0], __uint_as_float(c0[i]), __uint_as_float(c0[i + 1]));
+            pm[1] = fmax3(pm[1], __uint_as_float(c1[i]), __uint_as_float(c1[i + 1]));
           }
         } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            if (i <= r) pm[0] = fmaxf(pm[0], __uint_as_float(u0[i]));
-            if (32 + i <= r) pm[1] = fmaxf(pm[1], __uint_as_float(u1[i]));
+            if (i <= r) pm[0] = fmaxf(pm[0], __uint_as_float(c0[i]));
+            if (32 + i <= r) pm[1] = fmaxf(pm[1], __uint_as_float(c1[i]));
           }
         }
-      }
-      tmem_ld32(tS + 64, v0);
-      tmem_ld32(tS + 96, v1);
-      tmem_ld_wait();
-      if (!diag) {
+        tmem_ld_wait_regs(c2);
+        tmem_ld_wait_regs(c3);
+        if (!diag) {
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          pm[2] = fmax3(pm[2], __uint_as_float(v0[i]), __uint_as_float(v0[i + 1]));
-          pm[3] = fmax3(pm[3], __uint_as_float(v1[i]), __uint_as_float(v1[i + 1]));
-        }
-      } else {
+          for (int i = 0; i < 32; i += 2) {
+            pm[2] = fmax3(pm[2], __uint_as_float(c2[i]), __uint_as_float(c2[i + 1]));
+            pm[3] = fmax3(pm[3], __uint_as_float(c3[i]), __uint_as_float(c3[i + 1]));
+          }
+        } else {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          if (64 + i <= r) pm[2] = fmaxf(pm[2], __uint_as_float(v0[i]));
-          if (96 + i <= r) pm[3] = fmaxf(pm[3], __uint_as_float(v1[i]));
+          for (int i = 0; i < 32; ++i) {
+            if (64 + i <= r) pm[2] = fmaxf(pm[2], __uint_as_float(c2[i]));
+            if (96 + i <= r) pm[3] = fmaxf(pm[3], __uint_as_float(c3[i]));
+          }
         }
       }
       const float tmax = fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])) * a.scale_log2;
@@ -301,21 +302,25 @@ __global__ void __launch_bounds__(320, 1) prefill_attn_kernel(const __grid_const
         l *= alpha;
         m = mn;
       }
-      // P over S: keys [0, 64) are read again (P of a 32-key chunk only overwrites
-      // columns whose scores this thread has already read)
+      // P over S, 32 keys at a time, the next chunk's scores read while this chunk's
+      // P is computed (P of a chunk only overwrites columns already read)
       const uint64_t nm2 = f2_pack(-m, -m);
       uint64_t ls = 0ull;
       {
-        uint32_t u[32];
-        tmem_ld32(tS, u);
-        tmem_ld_wait();
-        ls = fadd2(ls, p_chunk(u, 0, diag, nm2));
-        tmem_ld32(tS + 32, u);
-        tmem_ld_wait();
-        ls = fadd2(ls, p_chunk(u, 32, diag, nm2));
+        uint32_t ua[32], ub[32];
+        tmem_ld32(tS, ua);
+        tmem_ld_wait_regs(ua);
+        tmem_ld32(tS + 32, ub);
+        ls = fadd2(ls, p_chunk(ua, 0, diag, nm2));
+        tmem_ld_wait_regs(ub);
+        tmem_ld32(tS + 64, ua);
+        ls = fadd2(ls, p_chunk(ub, 32, diag, nm2));
+        tmem_ld_wait_regs(ua);
+        tmem_ld32(tS + 96, ub);
+        ls = fadd2(ls, p_chunk(ua, 64, diag, nm2));
+        tmem_ld_wait_regs(ub);
+        ls = fadd2(ls, p_chunk(ub, 96, diag, nm2));
       }
-      ls = fadd2(ls, p_chunk(v0, 64, diag, nm2));
-      ls = fadd2(ls, p_chunk(v1, 96, diag, nm2));
       {
         float s0, s1;
         f2_unpack(ls, s0, s1);
