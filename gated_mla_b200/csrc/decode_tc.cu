@@ -6,20 +6,26 @@
 //   O_lat     = sum_s softmax(z)_s c_s              (weighted sum in latent space)
 //   o^(h)     = W_v^(h) O_lat;   out = sigmoid(g) ⊙ o   (W_v absorbed on the output side)
 //
-// Kernels, in launch order:
-//   1. decode_plan      split the cached tokens of all sequences into equal
-//                       per-CTA ranges of 128-token tiles (segments).
-//   2. decode_absorb    q_lat = W_k^T q (times scale*log2 e), bf16, with q^R appended.
-//   3. decode_attn      per (CTA range, head group): TMA streams the latent rows
-//                       through a ring of 16 KB boxes; tcgen05 computes
-//                       S^T = C Q_lat^T (M = 128 tokens, N = heads) into TMEM; four
-//                       softmax warps turn S^T into P (online softmax, fp32,
-//                       rescaling only when a running max grows by > 2^8); tcgen05
-//                       accumulates O^T = C^T P^T (M = 128 latent dims, N = heads)
-//                       in TMEM; at a segment end the partial (O, m, l) goes out.
-//   4. decode_merge     merges the partials of each (sequence, head) by their
-//                       log-sum-exp weights, applies W_v and the sigmoid gate and
-//                       writes the gated head outputs once.
+// Kernels, in launch order (the W_v product with the gate is a GEMM of gemm_tc.cu):
+//   1. decode_absorb_plan  q_lat = W_k^T q (times scale*log2 e), bf16, with q^R
+//                       appended; its last block splits the cached tokens of all
+//                       sequences into equal per-CTA ranges of 128-token tiles
+//                       (segments).
+//   2. decode_attn      per (CTA range, head group of HG heads): TMA streams the
+//                       latent rows through a ring of 16 KB boxes (128 tokens x 64
+//                       latent dims) in pairs, one full and one empty barrier per
+//                       pair; tcgen05 computes S^T = C Q_lat^T (M = 128 tokens,
+//                       N = HG) into one of two TMEM buffers; the softmax warps (four,
+//                       or eight as two head slices when HG >= 32) turn S^T into P
+//                       (online softmax in fp32, rescaling only when a running max
+//                       grows by > 2^8) and store P MN-major in shared memory;
+//                       tcgen05 accumulates O^T = C^T P^T (M = 128 latent dims,
+//                       N = HG) in TMEM. While the softmax works on a tile, the MMA
+//                       warp issues the score MMAs of the next tile's pairs that have
+//                       landed. At a segment end the partial (O, m, l) goes out.
+//   3. decode_merge     merges the partials of each (sequence, head) by their
+//                       log-sum-exp weights into O_lat (bf16 [H, B, d_c]), which the
+//                       W_v GEMM turns into the gated head outputs.
 #include "common.cuh"
 #include "internal.h"
 #include "ptx.cuh"

@@ -14,7 +14,9 @@
 //   kSwap = false (many tokens): MMA M = 128 token rows, N = BN weight rows.
 // Roles: warp 0 issues TMA loads into a ring of shared-memory stages, warp 1
 // allocates TMEM and one thread issues the MMAs, warps 2..5 drain the fp32
-// accumulator from TMEM and run the epilogue. Every wait is bounded.
+// accumulator from TMEM and run the epilogue. Every wait is bounded. In the
+// many-token orientation two CTAs share an SM, so that one CTA's epilogue runs
+// while the other's MMAs keep the tensor pipe busy.
 #include "common.cuh"
 #include "internal.h"
 #include "ptx.cuh"
