@@ -683,19 +683,26 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(DecodeArgs a) {
     for (int i = threadIdx.x; i < a.n_gemm_tiles; i += blockDim.x) a.gemm_counters[i] = 0;
   const int s0 = a.seq_first_seg[b], s1 = a.seq_first_seg[b + 1];
   const int64_t base = static_cast<int64_t>(hg) * a.max_seg;
-  float mx = -__int_as_float(0x7f800000);
-  for (int s = s0; s < s1; ++s) mx = fmaxf(mx, a.ml_part[((base + s) * a.HG + hl) * 2]);
-  float l = 0.f;
+  // one pass over the segments, rescaling the running sums when the max grows
+  // (every iteration's loads are independent of the previous ones)
+  float mx = -__int_as_float(0x7f800000), l = 0.f;
   float acc[kDc / 128];
 #pragma unroll
   for (int j = 0; j < kDc / 128; ++j) acc[j] = 0.f;
   for (int s = s0; s < s1; ++s) {
     const float* ml = a.ml_part + ((base + s) * a.HG + hl) * 2;
-    const float w = ex2_approx(ml[0] - mx);
-    l = fmaf(w, ml[1], l);
     const float* op = a.o_part + ((base + s) * a.HG + hl) * kDc;
+    const float ms = ml[0], ls = ml[1];
+    float o[kDc / 128];
 #pragma unroll
-    for (int j = 0; j < kDc / 128; ++j) acc[j] = fmaf(w, __ldcg(op + j * 128 + threadIdx.x), acc[j]);
+    for (int j = 0; j < kDc / 128; ++j) o[j] = __ldcg(op + j * 128 + threadIdx.x);
+    const float mn = fmaxf(mx, ms);
+    const float a_old = (mx == -__int_as_float(0x7f800000)) ? 0.f : ex2_approx(mx - mn);
+    const float a_new = (ms == -__int_as_float(0x7f800000)) ? 0.f : ex2_approx(ms - mn);
+    l = l * a_old + ls * a_new;
+#pragma unroll
+    for (int j = 0; j < kDc / 128; ++j) acc[j] = acc[j] * a_old + o[j] * a_new;
+    mx = mn;
   }
   const float inv = (s1 > s0 && l > 0.f) ? 1.f / l : 0.f;
   __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.olat) + (static_cast<int64_t>(h) * a.B + b) * kDc;
