@@ -253,6 +253,19 @@ def work_unit(w):
     return (1e9, "GB/s") if w.mode == "decode" else (1e12, "TFLOP/s")
 
 
+def job_throughput(local_ms, world, units_per_step, steps, scale, dist=None, device="cpu"):
+    """Whole-job throughput of `world` replicas: every rank processed `units_per_step`
+    units per step for `steps` steps; the job time is the slowest rank's (an
+    all-reduce MAX of the ranks' own device times when world > 1). Returns
+    (value in units/s / scale, max_ms)."""
+    import torch
+    t = torch.tensor([float(local_ms)], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    max_ms = float(t.item())
+    return world * units_per_step * steps / (max_ms / 1e3) / scale, max_ms
+
+
 def run_reference(args):
     import synth
     if int(os.environ.get("RANK", "0")) != 0:
@@ -445,11 +458,7 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     total_ms = sum(a.elapsed_time(b) for a, b in zip(ev0, ev1))
-    tt = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-    max_total_ms = float(tt.item())
-    value = world * run.work * K / (max_total_ms / 1e3) / scale
+    value, max_total_ms = job_throughput(total_ms, world, run.work, K, scale, dist, dev)
     run.model.sync_status()
 
     # per-kernel times: the step captured with the library's event records inside
@@ -511,10 +520,7 @@ def run_ours(args):
         e1[i].record(stream)
     torch.cuda.synchronize()
     e2e_ms = sum(a.elapsed_time(b) for a, b in zip(e0, e1))
-    et = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(et, op=dist.ReduceOp.MAX)
-    e2e_value = world * run.work * K / (float(et.item()) / 1e3) / scale
+    e2e_value, _ = job_throughput(e2e_ms, world, run.work, K, scale, dist, dev)
     run.model.sync_status()
 
     cpu = None
