@@ -63,7 +63,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
-                    choices=["decode_b32", "decode_long_rope", "decode_paged_head", "prefill_b4_s4096",
+                    choices=["decode_b32", "decode_long_rope", "decode_paged_head", "prefill_b4_s4096", "prefill_b1_s4096_h16",
                              "tiny_prefill_f32"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle CPU baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")

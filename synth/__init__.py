@@ -15,6 +15,8 @@ Workloads (sizes as named in the problem statement of Gated MLA):
                          lengths uniform in [1024, 8192], bf16.
 * ``prefill_b4_s4096``   batch 4, seq 4096, d_model 7168, H 64, d_h 128, d_c 512,
                          gate bias N(0, 2), bf16.
+* ``prefill_b1_s4096_h16`` batch 1, seq 4096, d_model 2048, H 16 (else as prefill_b4_s4096):
+  a reduced prefill for full ncu captures.
 * ``decode_long_rope``   batch 8, length 131072, d_model 7168, H 128, d_h 128,
                          d_c 512, decoupled RoPE d_R 64 (base 10000), bf16.
 * ``decode_paged_head``  batch 64 paged (page 64), lengths log-uniform in
@@ -87,6 +89,10 @@ WORKLOADS = {
     "prefill_b4_s4096": Workload(
         name="prefill_b4_s4096", mode="prefill", dtype="bf16", batch=4, seq_len=4096,
         d_model=7168, n_heads=64, d_h=128, d_c=512, gate_bias=True),
+    # a reduced prefill (one sequence, 16 heads) that a full ncu capture can replay quickly
+    "prefill_b1_s4096_h16": Workload(
+        name="prefill_b1_s4096_h16", mode="prefill", dtype="bf16", batch=1, seq_len=4096,
+        d_model=2048, n_heads=16, d_h=128, d_c=512, gate_bias=True),
     "decode_long_rope": Workload(
         name="decode_long_rope", mode="decode", dtype="bf16", batch=8, d_model=7168,
         n_heads=128, d_h=128, d_c=512, d_rope=64, rope_base=10000.0,
