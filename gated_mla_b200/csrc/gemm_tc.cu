@@ -404,6 +404,7 @@ __global__ void __launch_bounds__(192, kSwap ? 1 : 2) gemm_bf16_tc_kernel(const 
     // bytes on rank z's red_full); the owner sums the splits and stores. A CTA
     // leaves only after everything addressed to it has landed, and what it
     // sends comes from registers, so no second cluster barrier is needed.
+    __syncwarp();   // warps whose role ran on one lane arrive whole at the aligned barrier
     cluster_sync_all();
     float* recv = reinterpret_cast<float*>(smem);
     if (warp >= 2) {
