@@ -62,7 +62,9 @@ def params(inputs: dict) -> dict:
 
     ``inputs`` is the dict drawn by the seeded generator (or any dict with the
     same keys). Weight layouts are [out, in]: W_c [d_c, d_model],
-    W_kr [d_R, d_model], W_q [H*d_h, d_model], W_qr [H*d_R, d_model],
+    W_kr [d_R, d_model], W_q [H*d_h, d_model], W_qr [H*d_R, d_model]
+    (with a compressed query: W_dq [d_cq, d_model], W_uq [H*d_h, d_cq],
+    W_qr [H*d_R, d_cq] and no W_q),
     W_k / W_v [H, d_h, d_c], W_g [G, d_model], b_g [G], W_o [d_model, H*d_h].
     """
     w = inputs["workload"]
@@ -72,7 +74,8 @@ def params(inputs: dict) -> dict:
         "d_model": w.d_model, "gate_mode": w.gate_mode,
         "scale": w.softmax_scale, "rope_base": w.rope_base,
         "W_c": f(inputs["W_c"]), "W_kr": f(inputs.get("W_kr")),
-        "W_q": f(inputs["W_q"]), "W_qr": f(inputs.get("W_qr")),
+        "W_q": f(inputs.get("W_q")), "W_qr": f(inputs.get("W_qr")),
+        "W_dq": f(inputs.get("W_dq")), "W_uq": f(inputs.get("W_uq")),
         "W_k": f(inputs["W_k"]), "W_v": f(inputs["W_v"]),
         "W_g": f(inputs["W_g"]), "b_g": f(inputs.get("b_g")),
         "W_o": f(inputs["W_o"]),
@@ -138,8 +141,12 @@ def project_latent(p: dict, x: np.ndarray, positions: np.ndarray) -> dict:
 def project_query(p: dict, x: np.ndarray, positions: np.ndarray) -> dict:
     """What a token needs as a query:
 
-    * q  [T, H, d_h]     q^(h) = W_q^(h) x (reading: full-rank query)
-    * qR [T, H, d_R]     RoPE(W_qr^(h) x) at the token's position ([MLA-notes] §5.2)
+    * q  [T, H, d_h]     q^(h) = W_q^(h) x (reading: full-rank query), or with
+                         the low-rank query of [MLA-notes] §5.1
+                         c^Q = W_dq x (d_cq dims, returned as ``cq``), q = W_uq c^Q
+    * qR [T, H, d_R]     RoPE(W_qr^(h) x) at the token's position ([MLA-notes]
+                         §5.2); with the low-rank query RoPE(W_qr^(h) c^Q), as
+                         §5.2 writes q^R = RoPE(W^QR c^Q)
     * glogit [T, G]      W_g x (+ b_g): gate logits ([MLA-gate] §二 boxed
                          equation, per channel; [Gated-MLA concept] "Gating
                          Mechanism", per head with bias)
@@ -147,9 +154,14 @@ def project_query(p: dict, x: np.ndarray, positions: np.ndarray) -> dict:
     x = np.asarray(x, dtype=np.float64)
     T = x.shape[0]
     H, dh, dR = p["H"], p["d_h"], p["d_R"]
-    out = {"q": (x @ p["W_q"].T).reshape(T, H, dh)}
+    if p.get("W_dq") is not None:
+        q_in = x @ p["W_dq"].T                                     # c^Q [T, d_cq]
+        out = {"cq": q_in, "q": (q_in @ p["W_uq"].T).reshape(T, H, dh)}
+    else:
+        q_in = x
+        out = {"q": (x @ p["W_q"].T).reshape(T, H, dh)}
     if dR:
-        qr = (x @ p["W_qr"].T).reshape(T, H, dR)
+        qr = (q_in @ p["W_qr"].T).reshape(T, H, dR)
         out["qR"] = rope(qr, np.asarray(positions)[:, None], p["rope_base"])
     else:
         out["qR"] = np.zeros((T, H, 0))

@@ -22,9 +22,13 @@ Workloads (sizes as named in the problem statement of Gated MLA):
 * ``decode_paged_head``  batch 64 paged (page 64), lengths log-uniform in
                          [256, 32768], d_model 4096, H 32, d_h 128, d_c 512,
                          per-head gate with bias, bf16.
+* ``decode_long_rope_qc``, ``prefill_b4_s4096_qc``: the long-context decode
+                         and the batch-4 prefill with a low-rank query,
+                         d_cq 1536.
 
-Drawing order is fixed: x, W_c, W_kr, W_q, W_qr, W_k, W_v, W_g, b_g, W_o,
-lengths, page permutation, cache rows. Weights are N(0, 1/fan_in).
+Drawing order is fixed: x, W_c, W_kr, W_q (or W_dq, W_uq with a compressed
+query), W_qr, W_k, W_v, W_g, b_g, W_o, lengths, page permutation, cache rows.
+Weights are N(0, 1/fan_in).
 """
 from __future__ import annotations
 
@@ -59,6 +63,7 @@ class Workload:
     len_hi: int = 1
     paged: bool = False
     page_size: int = 64
+    d_cq: int = 0           # query low-rank compression width; 0 = full-rank query
 
     @property
     def softmax_scale(self) -> float:
@@ -101,6 +106,15 @@ WORKLOADS = {
         name="decode_paged_head", mode="decode", dtype="bf16", batch=64, d_model=4096,
         n_heads=32, d_h=128, d_c=512, gate_mode="head", gate_bias=True,
         len_law="loguniform", len_lo=256, len_hi=32768, paged=True, page_size=64),
+    # the long-context decode and the batch-4 prefill with a low-rank query of
+    # 1536 dims (the pages give the form, not a width)
+    "decode_long_rope_qc": Workload(
+        name="decode_long_rope_qc", mode="decode", dtype="bf16", batch=8, d_model=7168,
+        n_heads=128, d_h=128, d_c=512, d_rope=64, rope_base=10000.0,
+        len_law="fixed", len_lo=131072, len_hi=131072, d_cq=1536),
+    "prefill_b4_s4096_qc": Workload(
+        name="prefill_b4_s4096_qc", mode="prefill", dtype="bf16", batch=4, seq_len=4096,
+        d_model=7168, n_heads=64, d_h=128, d_c=512, gate_bias=True, d_cq=1536),
 }
 
 
@@ -176,7 +190,9 @@ def generate(w: Workload, seed: int = 0, lengths: Optional[np.ndarray] = None) -
                (prefill: all prompt tokens, packed by sequence; decode: the one
                new token per sequence)
     ``W_c``    [d_c, d_model]        ``W_kr`` [d_R, d_model] or None
-    ``W_q``    [H*d_h, d_model]      ``W_qr`` [H*d_R, d_model] or None
+    ``W_q``    [H*d_h, d_model] (None with a compressed query)
+    ``W_dq``   [d_cq, d_model], ``W_uq`` [H*d_h, d_cq] (compressed query only, else None)
+    ``W_qr``   [H*d_R, d_model] or [H*d_R, d_cq] with a compressed query, or None
     ``W_k``    [H, d_h, d_c]         ``W_v``  [H, d_h, d_c]
     ``W_g``    [G, d_model]          ``b_g``  [G] or None   (G = H*d_h or H)
     ``W_o``    [d_model, H*d_h]
@@ -200,8 +216,17 @@ def generate(w: Workload, seed: int = 0, lengths: Optional[np.ndarray] = None) -
     out["x"] = rnd(_normal(rng, (n_tok, dm), 1.0))
     out["W_c"] = rnd(_normal(rng, (dc, dm), 1.0 / math.sqrt(dm)))
     out["W_kr"] = rnd(_normal(rng, (dr, dm), 1.0 / math.sqrt(dm))) if dr else None
-    out["W_q"] = rnd(_normal(rng, (H * dh, dm), 1.0 / math.sqrt(dm)))
-    out["W_qr"] = rnd(_normal(rng, (H * dr, dm), 1.0 / math.sqrt(dm))) if dr else None
+    dcq = w.d_cq
+    if dcq:
+        # compressed query: c^Q = W_dq x, q = W_uq c^Q, q^R from c^Q (fan-in d_cq)
+        out["W_q"] = None
+        out["W_dq"] = rnd(_normal(rng, (dcq, dm), 1.0 / math.sqrt(dm)))
+        out["W_uq"] = rnd(_normal(rng, (H * dh, dcq), 1.0 / math.sqrt(dcq)))
+    else:
+        out["W_q"] = rnd(_normal(rng, (H * dh, dm), 1.0 / math.sqrt(dm)))
+        out["W_dq"] = out["W_uq"] = None
+    q_in = dcq or dm
+    out["W_qr"] = rnd(_normal(rng, (H * dr, q_in), 1.0 / math.sqrt(q_in))) if dr else None
     out["W_k"] = rnd(_normal(rng, (H, dh, dc), 1.0 / math.sqrt(dc)))
     out["W_v"] = rnd(_normal(rng, (H, dh, dc), 1.0 / math.sqrt(dc)))
     out["W_g"] = rnd(_normal(rng, (G, dm), 1.0 / math.sqrt(dm)))

@@ -58,8 +58,12 @@ def brute_prefill(inp):
     w = inp["workload"]
     H, dh, dR = w.n_heads, w.d_h, w.d_rope
     X = inp["x"].astype(float).tolist()
-    Wc, Wq, Wk, Wv, Wg, Wo = (np.asarray(inp[k], float).tolist() for k in
-                              ("W_c", "W_q", "W_k", "W_v", "W_g", "W_o"))
+    Wc, Wk, Wv, Wg, Wo = (np.asarray(inp[k], float).tolist() for k in ("W_c", "W_k", "W_v", "W_g", "W_o"))
+    compressed = inp.get("W_dq") is not None
+    if compressed:   # [MLA-notes] §5.1 c^Q = W^DQ h, q = W^UQ c^Q; §5.2 q^R = RoPE(W^QR c^Q)
+        Wdq, Wuq = np.asarray(inp["W_dq"], float).tolist(), np.asarray(inp["W_uq"], float).tolist()
+    else:
+        Wq = np.asarray(inp["W_q"], float).tolist()
     bg = np.asarray(inp["b_g"], float).tolist() if inp["b_g"] is not None else None
     Wkr = np.asarray(inp["W_kr"], float).tolist() if dR else None
     Wqr = np.asarray(inp["W_qr"], float).tolist() if dR else None
@@ -74,8 +78,9 @@ def brute_prefill(inp):
         kr = [_rot(_mv(Wkr, x), s, w.rope_base) for s, x in enumerate(xs)] if dR else None
         for t in range(L):
             x = xs[t]
-            qfull = _mv(Wq, x)
-            qrfull = _mv(Wqr, x) if dR else None
+            q_in = _mv(Wdq, x) if compressed else x
+            qfull = _mv(Wuq, q_in) if compressed else _mv(Wq, x)
+            qrfull = _mv(Wqr, q_in) if dR else None
             o_cat = []
             for h in range(H):
                 q = qfull[h * dh:(h + 1) * dh]
@@ -116,6 +121,33 @@ def test_bruteforce_prefill(d_rope, gate_mode):
     got = oracle.prefill(p, inp["x"], inp["lengths"])["y"]
     ref = brute_prefill(inp)
     np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("d_rope", [0, 2])
+def test_bruteforce_prefill_compressed_query(d_rope):
+    inp = tiny(d_rope=d_rope, d_cq=3)
+    assert inp["W_q"] is None and inp["W_dq"].shape == (3, 6) and inp["W_uq"].shape == (6, 3)
+    if d_rope:
+        assert inp["W_qr"].shape == (2 * 2, 3)     # q^R is read from c^Q
+    p = oracle.params(inp)
+    got = oracle.prefill(p, inp["x"], inp["lengths"])["y"]
+    np.testing.assert_allclose(got, brute_prefill(inp), rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("d_rope", [0, 2])
+def test_compressed_query_equals_full_rank_with_the_product_weight(d_rope):
+    """q = W_uq (W_dq x) is the full-rank query of W_q = W_uq W_dq, and
+    q^R = RoPE(W_qr (W_dq x)) the one of W_qr W_dq: the two oracle paths agree."""
+    inp = tiny(d_rope=d_rope, d_cq=4)
+    p = oracle.params(inp)
+    full = dict(p, W_q=p["W_uq"] @ p["W_dq"], W_dq=None, W_uq=None)
+    if d_rope:
+        full["W_qr"] = p["W_qr"] @ p["W_dq"]
+    a = oracle.prefill(p, inp["x"], inp["lengths"])
+    b = oracle.prefill(full, inp["x"], inp["lengths"])
+    for k in ("q", "qR", "o", "y"):
+        np.testing.assert_allclose(a[k], b[k], rtol=1e-12, atol=1e-13, err_msg=k)
+    np.testing.assert_allclose(a["cq"], np.asarray(inp["x"], float) @ p["W_dq"].T, rtol=1e-15)
 
 
 def test_two_token_closed_form():
@@ -363,6 +395,41 @@ def test_gate_never_changes_attention_weights():
 
 
 # ---------------------------------------------------------------------------
+# subset evaluation: the large-case parity tests ask the oracle for a few rows,
+# sequences or heads; each answer must equal the matching slice of the full one
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("d_rope", [0, 2])
+def test_prefill_row_subset_equals_full_rows(d_rope):
+    inp = tiny(d_rope=d_rope, lengths=(5, 7, 4))
+    p = oracle.params(inp)
+    full = oracle.prefill(p, inp["x"], inp["lengths"])
+    rows = {0: [4, 0, 2], 1: [6], 2: []}
+    sub = oracle.prefill(p, inp["x"], inp["lengths"], rows=rows)
+    want = np.array([0, 2, 4, 5 + 6])
+    assert np.array_equal(sub["index"], want)
+    # equal up to the summation order BLAS picks for a different number of rows
+    for k in ("q", "qR", "glogit", "o", "o_tilde", "gated", "y"):
+        np.testing.assert_allclose(sub[k], full[k][want], rtol=1e-13, atol=1e-15, err_msg=k)
+    # the whole cache side is always evaluated in full
+    np.testing.assert_array_equal(sub["c"], full["c"])
+
+
+@pytest.mark.parametrize("absorbed", [False, True])
+def test_decode_sequence_and_head_subsets_equal_full(absorbed):
+    d = tiny_decode(d_rope=2, lens=(1, 4, 7, 3))
+    p = oracle.params(d)
+    full = oracle.decode(p, d["x"], d["past"], absorbed=absorbed)
+    seqs, heads = [3, 1], [1]
+    sub = oracle.decode(p, d["x"], d["past"], seqs=seqs, heads=heads, absorbed=absorbed)
+    np.testing.assert_allclose(sub["o"], full["o"][np.ix_(seqs, heads)], rtol=1e-13, atol=1e-15)
+    assert "y" not in sub   # y needs every head
+    sub = oracle.decode(p, d["x"], d["past"], seqs=seqs, absorbed=absorbed)
+    for k in ("o", "o_tilde", "gated", "y"):
+        np.testing.assert_allclose(sub[k], full[k][seqs], rtol=1e-13, atol=1e-15, err_msg=k)
+
+
+# ---------------------------------------------------------------------------
 # printed numbers ([MLA-notes] §5.3, §7, 题1, 题5)
 # ---------------------------------------------------------------------------
 
@@ -476,3 +543,52 @@ def test_planted_mistake_is_caught(name, monkeypatch):
     monkeypatch.setattr(core, attr, new)
     monkeypatch.setattr(oracle, attr, new, raising=False)
     assert _run_all_pins() >= 1, f"planted mistake {name} passed every pin"
+
+
+# ---------------------------------------------------------------------------
+# the rescale-path GPU inputs have teeth: simulated on the CPU with the
+# kernels' tiling and raise rule, dropping the rescale of the partial output
+# moves the result far outside the bf16 tolerance
+# ---------------------------------------------------------------------------
+
+def _online_latent(z2, C, tile=128, raise_by=8.0, rescale=True):
+    """sum_s 2^(z2_s - m) c_s / sum_s 2^(z2_s - m) by tiles, raising the running
+    max m only by more than raise_by; with rescale=False the accumulated sum is
+    not multiplied by 2^(m_old - m_new) when m rises (the mistake to expose)."""
+    m, l, O = -np.inf, 0.0, np.zeros(C.shape[1])
+    for t0 in range(0, len(z2), tile):
+        zt, Ct = z2[t0:t0 + tile], C[t0:t0 + tile]
+        if t0 == 0 or zt.max() > m + raise_by:
+            mn = max(m, zt.max())
+            alpha = 0.0 if m == -np.inf else 2.0 ** (m - mn)
+            l *= alpha
+            if rescale:
+                O *= alpha
+            m = mn
+        p = 2.0 ** (zt - m)
+        l += p.sum()
+        O += p @ Ct
+    return O / l
+
+
+def test_peaked_decode_input_needs_the_rescale():
+    import sys
+    sys.path.insert(0, os.path.dirname(__file__))
+    from gpu_pipeline import small_decode
+    from rescale_inputs import decode_scores_log2, plant_decode
+    inp = small_decode("decode_b32", 2, [2000, 1500])
+    inp = plant_decode(inp, [(b, 300 + 61 * h, h, 16.0) for b in range(2) for h in range(16)])
+    dc = inp["workload"].d_c
+    worst = 0.0
+    for b in range(2):
+        z = decode_scores_log2(inp, b)
+        p = oracle.params(inp)
+        c_new = oracle.project_latent(p, np.asarray(inp["x"], float)[b:b + 1], np.array([len(inp["past"][b])]))["c"]
+        C = np.concatenate([np.asarray(inp["past"][b], float)[:, :dc], c_new])
+        for h in range(z.shape[0]):
+            exact = oracle.core._softmax_rows((z[h] * math.log(2.0))[None])[0] @ C
+            good = _online_latent(z[h], C)
+            np.testing.assert_allclose(good, exact, rtol=1e-9, atol=1e-12)
+            bad = _online_latent(z[h], C, rescale=False)
+            worst = max(worst, np.linalg.norm(bad - exact) / np.linalg.norm(exact))
+    assert worst > 1.0, worst
