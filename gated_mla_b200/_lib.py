@@ -37,12 +37,13 @@ class gmla_config(ctypes.Structure):
         ("softmax_scale", ctypes.c_float),
         ("rope_base", ctypes.c_float),
         ("dtype", ctypes.c_int32),
+        ("d_cq", ctypes.c_int32),
     ]
 
 
 class gmla_weights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
-                ("W_c", "W_kr", "W_q", "W_qr", "W_k", "W_v", "W_g", "b_g", "W_o")]
+                ("W_c", "W_kr", "W_q", "W_qr", "W_k", "W_v", "W_g", "b_g", "W_o", "W_dq", "W_uq")]
 
 
 class gmla_cache(ctypes.Structure):
@@ -92,6 +93,7 @@ def _load() -> ctypes.CDLL:
         "gmla_last_error": (ctypes.c_char_p, []),
         "gmla_version": (ctypes.c_char_p, []),
         "gmla_launch_count": (ctypes.c_uint64, []),
+        "gmla_test_stall_next_decode": (st, [I]),
         "gmla_profile_enable": (st, [I]),
         "gmla_profile_count": (I, []),
         "gmla_profile_get": (st, [I, ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(ctypes.c_float)]),
@@ -159,6 +161,10 @@ def gmla_clear_status(ws, stream):
 
 def gmla_sync_status(ws, stream):
     return lib.gmla_sync_status(ws, stream)
+
+
+def gmla_test_stall_next_decode(enable):
+    return lib.gmla_test_stall_next_decode(1 if enable else 0)
 
 
 def gmla_launch_count():

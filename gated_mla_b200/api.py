@@ -59,7 +59,7 @@ class GatedMLA:
     def __init__(self, *, d_model: int, n_heads: int, d_h: int, d_c: int, d_rope: int = 0,
                  gate_mode: str = "channel", softmax_scale: Optional[float] = None,
                  rope_base: float = 10000.0, dtype: torch.dtype = torch.bfloat16,
-                 weights: dict):
+                 weights: dict, d_cq: int = 0):
         self.dtype = dtype
         self.cfg = L.gmla_config()
         self.cfg.d_model, self.cfg.n_heads, self.cfg.d_h, self.cfg.d_c, self.cfg.d_rope = (
@@ -69,9 +69,10 @@ class GatedMLA:
         self.cfg.softmax_scale = softmax_scale if softmax_scale else 1.0 / math.sqrt(d_h + d_rope)
         self.cfg.rope_base = rope_base
         self.cfg.dtype = _DT[dtype]
+        self.cfg.d_cq = d_cq
         self.weights = dict(weights)
         self.w = L.gmla_weights()
-        for k in ("W_c", "W_kr", "W_q", "W_qr", "W_k", "W_v", "W_g", "b_g", "W_o"):
+        for k in ("W_c", "W_kr", "W_q", "W_qr", "W_k", "W_v", "W_g", "b_g", "W_o", "W_dq", "W_uq"):
             setattr(self.w, k, _p(self.weights.get(k)))
         self._ws = {}
 

@@ -229,9 +229,10 @@ struct DecSmem {
   uint64_t rope_full, rope_empty;
   uint64_t q_full, q_empty;
   uint64_t s_full, p_full, o_done, o_free, drain;
+  uint64_t never;               // completed by nothing (the stall test hook waits on it)
   uint32_t tmem;
   int abort;
-  int vote[2];
+  int vote[3];
   int red[2][4][64];
   float lred[4][64];
   float mfin[64];
@@ -291,8 +292,9 @@ __global__ void __launch_bounds__(64 + 128 * (HG >= 32 ? 2 : 1), 1) decode_attn_
     mbar_init(&sm->o_done, 1);
     mbar_init(&sm->o_free, 128 * C::kSG);
     mbar_init(&sm->drain, 1);
+    mbar_init(&sm->never, 1);
     sm->abort = 0;
-    sm->vote[0] = sm->vote[1] = 0;
+    sm->vote[0] = sm->vote[1] = sm->vote[2] = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -398,6 +400,13 @@ __global__ void __launch_bounds__(64 + 128 * (HG >= 32 ? 2 : 1), 1) decode_attn_
       uint32_t npair = 0, nrope = 0, ntile = 0, nseg = 0;
       int early = 0;   // pairs of this tile whose score MMAs were issued during the previous tile
       bool ok = true;
+      if (a.test_stall && g == 0 && hg == 0) {
+        // Test hook: the first CTA's MMA thread waits on a barrier that nothing
+        // completes, as it would behind a stalled copy. The bounded wait runs out,
+        // raises the block's abort flag and reports a timeout in the status word;
+        // every role then leaves through its abort path (copies drained, TMEM freed).
+        ok = mbar_wait(&sm->never, 0, abort_flag, a.status);
+      }
       // Descriptors are built once; an operand's descriptor is the base one plus its
       // byte offset / 16 (the start-address field cannot carry: shared addresses < 256 KB).
       const uint64_t dRing = sdesc_sw128(ring_a, 16, 1024), dQ = sdesc_sw128(q_a, 16, 1024);
@@ -522,12 +531,16 @@ __global__ void __launch_bounds__(64 + 128 * (HG >= 32 ? 2 : 1), 1) decode_attn_
 #pragma unroll
           for (int j = 0; j < 16; ++j) need |= x[j] > m[c + j] + 8.f;
         }
-        // block-wide vote among the softmax threads
+        // block-wide vote among the softmax threads, one of three slots per tile:
+        // after tile n's barrier the slot of tile n - 1 (= n + 2 mod 3) is cleared;
+        // its readers finished before this barrier and its next writers (tile n + 2)
+        // come after the barrier of tile n + 1, so no vote can be erased
         const int par = ntile & 1;
-        if (__any_sync(0xffffffffu, need) && lane == 0) atomicOr(&sm->vote[par], 1);
+        const int vslot = static_cast<int>(ntile % 3u);
+        if (__any_sync(0xffffffffu, need) && lane == 0) atomicOr(&sm->vote[vslot], 1);
         asm volatile("bar.sync 1, %0;" ::"n"(128 * SG) : "memory");
-        const bool need_all = sm->vote[par] != 0;
-        if (ltid == 0) sm->vote[par ^ 1] = 0;
+        const bool need_all = sm->vote[vslot] != 0;
+        if (ltid == 0) sm->vote[(vslot + 2) % 3] = 0;
         if (need_all) {
 #pragma unroll
           for (int c = 0; c < HT; c += 16) {

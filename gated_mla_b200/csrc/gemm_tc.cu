@@ -266,7 +266,8 @@ __global__ void __launch_bounds__(192, kSwap ? 1 : 2) gemm_bf16_tc_kernel(const 
     }
     // Split-K epilogues meet at named barrier 2; a failed wait still walks the
     // same barriers (with its stores skipped) so the four warps stay in step.
-    const bool acc_ok = mbar_wait(acc_full, 0, abort_flag, a.status);
+    // warp-uniform: the TMEM loads below are warp-collective
+    const bool acc_ok = __all_sync(0xffffffffu, mbar_wait(acc_full, 0, abort_flag, a.status));
     if (acc_ok || kSwap) {
       tc_fence_after();
       if (kSwap) {
@@ -401,15 +402,18 @@ __global__ void __launch_bounds__(192, kSwap ? 1 : 2) gemm_bf16_tc_kernel(const 
     // completes, so their stage memory is idle and receives the partials:
     // recv[src split][row][cpr] fp32. Each split pushes the columns that rank
     // z owns straight from its accumulator to rank z (st.async, completing
-    // bytes on rank z's red_full); the owner sums the splits and stores. A CTA
-    // leaves only after everything addressed to it has landed, and what it
-    // sends comes from registers, so no second cluster barrier is needed.
+    // bytes on rank z's red_full); the owner sums the splits and stores.
+    // A second cluster barrier, split into an arrive after the sends and a wait
+    // before the block exits, keeps every CTA resident until all of its peers
+    // have issued what they send to it, also when an owner's wait for its
+    // partials gave up. Nothing between the two halves waits without a bound,
+    // so the final wait ends once every CTA has issued its sends.
     __syncwarp();   // warps whose role ran on one lane arrive whole at the aligned barrier
     cluster_sync_all();
     float* recv = reinterpret_cast<float*>(smem);
     if (warp >= 2) {
       const int q = warp & 3, r = q * 32 + lane;
-      const bool acc_ok = !*abort_flag;
+      const bool acc_ok = __all_sync(0xffffffffu, !*abort_flag);
       tc_fence_after();
 #pragma unroll 1
       for (int c0 = 0; c0 < BN; c0 += 16) {
@@ -427,6 +431,10 @@ __global__ void __launch_bounds__(192, kSwap ? 1 : 2) gemm_bf16_tc_kernel(const 
           st_async_v4(cluster_map(dst, z), x, cluster_map(smem_u32(red_full), z));
         }
       }
+    }
+    cluster_arrive_release();   // every thread: this CTA's sends are issued
+    if (warp >= 2) {
+      const int q = warp & 3, r = q * 32 + lane;
       if (own_cols > 0) {
         const bool got = mbar_wait_cluster(red_full, 0, abort_flag, a.status);
         const int col0 = static_cast<int>(rank) * cpr;
@@ -491,6 +499,7 @@ __global__ void __launch_bounds__(192, kSwap ? 1 : 2) gemm_bf16_tc_kernel(const 
         }
       }
     }
+    cluster_wait_acquire();   // no CTA leaves while a peer may still send into it
   }
 
   // one lane of a warp ran a role alone: reconverge before the block-wide barrier

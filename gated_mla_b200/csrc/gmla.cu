@@ -85,7 +85,7 @@ const char* status_str(gmla_status s) {
 
 gmla_status check_cfg(const gmla_config* c) {
   if (!c) return fail(GMLA_ERR_INVALID_ARG, "config is NULL");
-  if (c->d_model <= 0 || c->n_heads <= 0 || c->d_h <= 0 || c->d_c <= 0 || c->d_rope < 0)
+  if (c->d_model <= 0 || c->n_heads <= 0 || c->d_h <= 0 || c->d_c <= 0 || c->d_rope < 0 || c->d_cq < 0)
     return fail(GMLA_ERR_INVALID_ARG, "non-positive dimension in config");
   if (c->d_rope % 2) return fail(GMLA_ERR_INVALID_ARG, "d_rope must be even (RoPE rotates pairs)");
   if (c->gate_mode != GMLA_GATE_CHANNEL && c->gate_mode != GMLA_GATE_HEAD)
@@ -95,6 +95,20 @@ gmla_status check_cfg(const gmla_config* c) {
     return fail(GMLA_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
   if (c->d_rope && !(c->rope_base > 1.f)) return fail(GMLA_ERR_INVALID_ARG, "rope_base must be > 1");
   return GMLA_OK;
+}
+
+// The same checks as check_cfg, without touching the thread's last error (for
+// the size queries, which return a status-free value).
+bool cfg_valid(const gmla_config* c) {
+  if (!c) return false;
+  if (c->d_model <= 0 || c->n_heads <= 0 || c->d_h <= 0 || c->d_c <= 0 || c->d_rope < 0 || c->d_cq < 0)
+    return false;
+  if (c->d_rope % 2) return false;
+  if (c->gate_mode != GMLA_GATE_CHANNEL && c->gate_mode != GMLA_GATE_HEAD) return false;
+  if (c->dtype != GMLA_BF16 && c->dtype != GMLA_FP32) return false;
+  if (!(c->softmax_scale > 0.f) || !std::isfinite(c->softmax_scale)) return false;
+  if (c->d_rope && !(c->rope_base > 1.f)) return false;
+  return true;
 }
 
 gmla_status check_ptr(const void* p, const char* name, bool required = true) {
@@ -171,21 +185,15 @@ std::vector<ProfRec> g_prof;
 size_t g_prof_used = 0;
 bool g_prof_open = false;
 std::atomic<uint64_t> g_launches{0};
-
-// K split of a swap-orientation GEMM (the splits reduce through a cluster).
-cudaError_t set_splits(GemmArgs& a, const SwapPlan& sp, uint8_t* ws, cudaStream_t st) {
-  (void)ws;
-  (void)st;
-  a.splits = sp.splits;
-  a.kb_per_split = sp.kb_per_split;
-  return cudaSuccess;
-}
+std::atomic<int> g_test_stall{0};   // armed by gmla_test_stall_next_decode
 
 }  // namespace
 
 namespace gmla {
 
 void set_last_error(const char* msg) { g_err = msg ? msg : ""; }
+
+int check_config(const ::gmla_config* c) { return check_cfg(c); }
 
 void prof_begin(cudaStream_t st, const char* name) {
   g_launches.fetch_add(1, std::memory_order_relaxed);
@@ -252,6 +260,11 @@ const char* gmla_version(void) { return "gmla 0.1.0 sm_100a"; }
 
 uint64_t gmla_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
+gmla_status gmla_test_stall_next_decode(int32_t enable) {
+  g_test_stall.store(enable ? 1 : 0);
+  return GMLA_OK;
+}
+
 gmla_status gmla_profile_enable(int32_t enable) {
   std::lock_guard<std::mutex> lk(g_prof_mu);
   g_prof_on = enable != 0;
@@ -277,21 +290,19 @@ gmla_status gmla_profile_get(int32_t i, const char** name, float* ms) {
   return GMLA_OK;
 }
 
-static int project_wtiles(const gmla_config* c) {
-  const int G = c->gate_mode == GMLA_GATE_CHANNEL ? c->n_heads * c->d_h : c->n_heads;
-  const int rows[5] = {c->d_c, c->d_rope, c->n_heads * c->d_h, c->n_heads * c->d_rope, G};
-  int t = 0;
-  for (int r : rows) t += (r + 127) / 128;
-  return t;
+// Bytes of the compressed query c^Q [T, d_cq] kept in the workspace (after the status word).
+static size_t cq_bytes(const gmla_config* c, int32_t T) {
+  if (c->d_cq <= 0) return 0;
+  return align256(static_cast<size_t>(T) * c->d_cq * (c->dtype == GMLA_FP32 ? 4 : 2));
 }
 
 size_t gmla_latent_project_workspace_size(const gmla_config* cfg, int32_t T) {
-  if (!cfg || T < 0 || cfg->dtype == GMLA_FP32 || T > 256) return 256;
-  return 256 + gemm_swap_plan(project_wtiles(cfg), T, cfg->d_model, num_sms()).ws_bytes;
+  if (!cfg_valid(cfg) || T < 0) return 256;
+  return 256 + cq_bytes(cfg, T);
 }
 
 size_t gmla_gate_out_workspace_size(const gmla_config* cfg, int32_t T) {
-  if (!cfg || T < 0) return 256;
+  if (!cfg_valid(cfg) || T < 0) return 256;
   const size_t es = cfg->dtype == GMLA_FP32 ? 4 : 2;
   size_t n = 256 + align256(static_cast<size_t>(T) * cfg->n_heads * cfg->d_h * es);
   if (cfg->dtype != GMLA_FP32 && T <= 256)
@@ -300,13 +311,13 @@ size_t gmla_gate_out_workspace_size(const gmla_config* cfg, int32_t T) {
 }
 
 size_t gmla_decode_workspace_size(const gmla_config* cfg, int32_t B) {
-  if (!cfg || B < 0) return 256;
+  if (!cfg_valid(cfg) || B < 0) return 256;
   if (cfg->dtype == GMLA_FP32) return 256;
   return decode_layout(B, cfg->n_heads, cfg->d_h, cfg->d_c, cfg->d_rope, num_sms()).total;
 }
 
 size_t gmla_prefill_workspace_size(const gmla_config* cfg, int32_t T, int32_t B) {
-  if (!cfg || T < 0 || B < 0) return 256;
+  if (!cfg_valid(cfg) || T < 0 || B < 0) return 256;
   const size_t es = cfg->dtype == GMLA_FP32 ? 4 : 2;
   const size_t kv = static_cast<size_t>(T) * cfg->n_heads * cfg->d_h * es;
   return 256 + 2 * align256(kv);
@@ -331,6 +342,83 @@ gmla_status gmla_sync_status(const void* workspace, void* stream) {
 }
 
 // ---------------------------------------------------------------------------
+}  // extern "C"
+
+namespace {
+
+struct ProjSeg {
+  const void* W;
+  int rows;
+  EpiSeg e;
+};
+
+// One projection GEMM: act [T, K] times the weight segments, each segment with
+// its own epilogue (tcgen05 kernel for bf16, CUDA-core kernel for fp32).
+gmla_status project_gemm(const gmla_config* cfg, const void* act, int T, int K, const ProjSeg* segs, int ns,
+                         const int32_t* positions, const int32_t* seq_ids, const CacheView& cv, int* status,
+                         cudaStream_t st, const char* name) {
+  const bool f32 = cfg->dtype == GMLA_FP32;
+  const double log2_base = cfg->d_rope ? std::log2(static_cast<double>(cfg->rope_base)) : 0.0;
+  if (f32) {
+    F32Args a{};
+    a.x = static_cast<const float*>(act);
+    a.T = T;
+    a.K = K;
+    a.n_seg = ns;
+    for (int i = 0; i < ns; ++i) {
+      a.W[i] = static_cast<const float*>(segs[i].W);
+      a.epi[i] = segs[i].e;
+      a.seg_rows[i] = segs[i].rows;
+    }
+    a.positions = positions;
+    a.seq_ids = seq_ids;
+    a.cache = cv;
+    a.log2_rope_base = log2_base;
+    a.status = status;
+    cudaError_t e = launch_gemm_f32(a, st);
+    return e == cudaSuccess ? GMLA_OK : cuda_fail(e, name);
+  }
+  if (K % 8) return fail(GMLA_ERR_UNSUPPORTED, "%s: the bf16 path needs an inner dimension %% 8 == 0", name);
+  int wtiles = 0;
+  for (int i = 0; i < ns; ++i) wtiles += (segs[i].rows + 127) / 128;
+  GemmArgs a{};
+  const bool swap = T <= 256;
+  const SwapPlan sp = gemm_swap_plan(wtiles, T, K, num_sms());
+  const int bn = swap ? sp.bn : 256;
+  const int wtile = gemm_weight_tile(swap, bn);
+  if (!make_tmap_2d(&a.act, act, K, T, static_cast<uint64_t>(K) * 2, 64, swap ? bn : 128, true))
+    return fail(GMLA_ERR_CUDA, "%s: tensor map for the activations failed", name);
+  a.seg_tile_begin[0] = 0;
+  for (int i = 0; i < ns; ++i) {
+    if (!make_tmap_2d(&a.wt[i], segs[i].W, K, segs[i].rows, static_cast<uint64_t>(K) * 2, 64, wtile, true))
+      return fail(GMLA_ERR_CUDA, "%s: tensor map for weight segment %d failed", name, i);
+    a.epi[i] = segs[i].e;
+    a.seg_rows[i] = segs[i].rows;
+    a.seg_tile_begin[i + 1] = a.seg_tile_begin[i] + (segs[i].rows + wtile - 1) / wtile;
+  }
+  a.n_seg = ns;
+  a.T = T;
+  a.K = K;
+  a.row_mode = 0;
+  a.positions = positions;
+  a.seq_ids = seq_ids;
+  a.cache = cv;
+  a.log2_rope_base = log2_base;
+  a.status = status;
+  if (swap) {
+    a.splits = sp.splits;
+    a.kb_per_split = sp.kb_per_split;
+  }
+  const int ttiles = swap ? sp.ttiles : (T + 127) / 128;
+  cudaError_t e = launch_gemm_bf16(a, swap, bn, ttiles, st, name);
+  return e == cudaSuccess ? GMLA_OK : cuda_fail(e, name);
+}
+
+}  // namespace
+
+extern "C" {
+
+// ---------------------------------------------------------------------------
 gmla_status gmla_latent_project(const gmla_config* cfg, const gmla_weights* w, const void* x, int32_t T,
                                 const int32_t* positions, const int32_t* seq_ids, const gmla_cache* cache,
                                 void* q_out, float* gate_logits, void* workspace, size_t workspace_bytes,
@@ -342,14 +430,21 @@ gmla_status gmla_latent_project(const gmla_config* cfg, const gmla_weights* w, c
   if (!workspace || workspace_bytes < gmla_latent_project_workspace_size(cfg, T))
     return fail(GMLA_ERR_WORKSPACE, "latent_project needs %zu workspace bytes",
                 gmla_latent_project_workspace_size(cfg, T));
+  GMLA_TRY(check_ptr(workspace, "workspace"));
   if (T == 0) return GMLA_OK;
+  const bool compressed = cfg->d_cq > 0;
   GMLA_TRY(check_ptr(x, "x"));
   GMLA_TRY(check_ptr(positions, "positions"));
   GMLA_TRY(check_ptr(seq_ids, "seq_ids"));
   GMLA_TRY(check_ptr(q_out, "q_out"));
   GMLA_TRY(check_ptr(gate_logits, "gate_logits"));
   GMLA_TRY(check_ptr(w->W_c, "W_c"));
-  GMLA_TRY(check_ptr(w->W_q, "W_q"));
+  if (compressed) {
+    GMLA_TRY(check_ptr(w->W_dq, "W_dq"));
+    GMLA_TRY(check_ptr(w->W_uq, "W_uq"));
+  } else {
+    GMLA_TRY(check_ptr(w->W_q, "W_q"));
+  }
   GMLA_TRY(check_ptr(w->W_g, "W_g"));
   if (cfg->d_rope) {
     GMLA_TRY(check_ptr(w->W_kr, "W_kr"));
@@ -362,73 +457,33 @@ gmla_status gmla_latent_project(const gmla_config* cfg, const gmla_weights* w, c
   const int dq = dh + dr;
   const CacheView cv = cache_view(cfg, cache);
   int* status = static_cast<int*>(workspace);
-
-  // segments of the weight dimension: [W_c | W_kr | W_q | W_qr | W_g]
-  struct Seg {
-    const void* W;
-    int rows;
-    EpiSeg e;
-  } segs[kMaxSeg];
-  int ns = 0;
   const bool f32 = cfg->dtype == GMLA_FP32;
+  void* cq = static_cast<uint8_t*>(workspace) + 256;   // c^Q [T, d_cq] when the query is compressed
+
+  // GEMM over x: [W_c | W_kr | W_q | W_qr | W_g], or [W_c | W_kr | W_dq | W_g] with a
+  // compressed query ("精读笔记 03" §5.1: c^Q = W^DQ h), whose second GEMM reads c^Q:
+  // [W_uq | W_qr] (q = W^UQ c^Q; §5.2: q^R = RoPE(W^QR c^Q)).
+  const EpiSeg e_q = plain_seg(q_out, static_cast<int64_t>(H) * dq, dh, dq, 0, f32, nullptr, false, false);
+  const EpiSeg e_qr = plain_seg(q_out, static_cast<int64_t>(H) * dq, dr, dq, dh, f32, nullptr, true, false);
+  ProjSeg segs[kMaxSeg];
+  int ns = 0;
   segs[ns++] = {w->W_c, dc, plain_seg(cache->data, row, 1 << 30, 0, 0, f32, nullptr, false, true)};
   if (dr) segs[ns++] = {w->W_kr, dr, plain_seg(cache->data, row, dr, 0, dc, f32, nullptr, true, true)};
-  segs[ns++] = {w->W_q, H * dh, plain_seg(q_out, static_cast<int64_t>(H) * dq, dh, dq, 0, f32, nullptr, false, false)};
-  if (dr)
-    segs[ns++] = {w->W_qr, H * dr, plain_seg(q_out, static_cast<int64_t>(H) * dq, dr, dq, dh, f32, nullptr, true, false)};
+  if (compressed) {
+    segs[ns++] = {w->W_dq, cfg->d_cq, plain_seg(cq, cfg->d_cq, 1 << 30, 0, 0, f32, nullptr, false, false)};
+  } else {
+    segs[ns++] = {w->W_q, H * dh, e_q};
+    if (dr) segs[ns++] = {w->W_qr, H * dr, e_qr};
+  }
   segs[ns++] = {w->W_g, G,
                 plain_seg(gate_logits, G, 1 << 30, 0, 0, true, cfg->gate_bias ? w->b_g : nullptr, false, false)};
-
-  if (f32) {
-    F32Args a{};
-    a.x = static_cast<const float*>(x);
-    a.T = T;
-    a.K = dm;
-    a.n_seg = ns;
-    for (int i = 0; i < ns; ++i) {
-      a.W[i] = static_cast<const float*>(segs[i].W);
-      a.epi[i] = segs[i].e;
-      a.seg_rows[i] = segs[i].rows;
-    }
-    a.positions = positions;
-    a.seq_ids = seq_ids;
-    a.cache = cv;
-    a.log2_rope_base = dr ? std::log2(static_cast<double>(cfg->rope_base)) : 0.0;
-    a.status = status;
-    cudaError_t e = launch_gemm_f32(a, st);
-    return e == cudaSuccess ? GMLA_OK : cuda_fail(e, "latent_project (fp32)");
-  }
-
-  if (dm % 8) return fail(GMLA_ERR_UNSUPPORTED, "bf16 path needs d_model %% 8 == 0");
-  GemmArgs a{};
-  const bool swap = T <= 256;
-  const SwapPlan sp = gemm_swap_plan(project_wtiles(cfg), T, dm, num_sms());
-  const int bn = swap ? sp.bn : 256;
-  const int wtile = gemm_weight_tile(swap, bn);
-  if (!make_tmap_2d(&a.act, x, dm, T, static_cast<uint64_t>(dm) * 2, 64, swap ? bn : 128, true))
-    return fail(GMLA_ERR_CUDA, "tensor map for x failed");
-  a.seg_tile_begin[0] = 0;
-  for (int i = 0; i < ns; ++i) {
-    if (!make_tmap_2d(&a.wt[i], segs[i].W, dm, segs[i].rows, static_cast<uint64_t>(dm) * 2, 64, wtile, true))
-      return fail(GMLA_ERR_CUDA, "tensor map for weight segment %d failed", i);
-    a.epi[i] = segs[i].e;
-    a.seg_rows[i] = segs[i].rows;
-    a.seg_tile_begin[i + 1] = a.seg_tile_begin[i] + (segs[i].rows + wtile - 1) / wtile;
-  }
-  a.n_seg = ns;
-  a.T = T;
-  a.K = dm;
-  a.row_mode = 0;
-  a.positions = positions;
-  a.seq_ids = seq_ids;
-  a.cache = cv;
-  a.log2_rope_base = dr ? std::log2(static_cast<double>(cfg->rope_base)) : 0.0;
-  a.status = status;
-  const int ttiles = swap ? sp.ttiles : (T + 127) / 128;
-  cudaError_t e = cudaSuccess;
-  if (swap) e = set_splits(a, sp, static_cast<uint8_t*>(workspace) + 256, st);
-  if (e == cudaSuccess) e = launch_gemm_bf16(a, swap, bn, ttiles, st, "gemm_project");
-  return e == cudaSuccess ? GMLA_OK : cuda_fail(e, "latent_project");
+  GMLA_TRY(project_gemm(cfg, x, T, dm, segs, ns, positions, seq_ids, cv, status, st, "gemm_project"));
+  if (!compressed) return GMLA_OK;
+  ProjSeg qsegs[2];
+  int nq = 0;
+  qsegs[nq++] = {w->W_uq, H * dh, e_q};
+  if (dr) qsegs[nq++] = {w->W_qr, H * dr, e_qr};
+  return project_gemm(cfg, cq, T, cfg->d_cq, qsegs, nq, positions, seq_ids, cv, status, st, "gemm_query_up");
 }
 
 // ---------------------------------------------------------------------------
@@ -525,6 +580,7 @@ gmla_status gmla_decode(const gmla_config* cfg, const gmla_weights* w, const voi
   a.G = L.G;
   a.max_seg = L.max_seg;
   a.q_scale = cfg->softmax_scale * 1.4426950408889634f;
+  a.test_stall = g_test_stall.exchange(0);
   a.olat = ws + L.off_olat;
   const SwapPlan& sp = L.gemm_plan;
   a.gemm_counters = nullptr;
@@ -730,9 +786,11 @@ gmla_status gmla_gate_out(const gmla_config* cfg, const gmla_weights* w, const v
   a.row_mode = 0;
   a.status = status;
   const int ttiles = swap ? sp.ttiles : (T + 127) / 128;
-  cudaError_t e = cudaSuccess;
-  if (swap) e = set_splits(a, sp, static_cast<uint8_t*>(workspace) + 256 + align256(static_cast<size_t>(T) * HD * 2), st);
-  if (e == cudaSuccess) e = launch_gemm_bf16(a, swap, bn, ttiles, st, "gemm_out");
+  if (swap) {
+    a.splits = sp.splits;
+    a.kb_per_split = sp.kb_per_split;
+  }
+  cudaError_t e = launch_gemm_bf16(a, swap, bn, ttiles, st, "gemm_out");
   return e == cudaSuccess ? GMLA_OK : cuda_fail(e, "gate_out");
 }
 

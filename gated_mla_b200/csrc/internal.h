@@ -7,7 +7,13 @@
 
 #include "common.cuh"
 
+struct gmla_config;
+
 namespace gmla {
+
+// Argument check of a configuration shared by the entry points (gmla.cu):
+// returns a gmla_status and sets the thread's last error when it fails.
+int check_config(const ::gmla_config* c);
 
 // Launches `kernel` with programmatic stream serialization: it may begin
 // while the previous kernel of the stream is still running, and calls
@@ -75,6 +81,7 @@ struct DecodeArgs {
   int32_t B, H, d_h, d_c, d_rope, gate_mode;
   int32_t HG, n_hg, G, max_seg;
   float q_scale;             // softmax_scale * log2(e), folded into the absorbed query
+  int32_t test_stall;        // test hook: the first CTA's MMA thread waits on a barrier nothing completes
 };
 
 struct DecodeLayout {

@@ -63,8 +63,11 @@ extern "C" GMLA_API gmla_status gmla_decode_noalloc(const gmla_config* cfg, cons
                                                     const float* gate_logits, const gmla_cache* cache,
                                                     const int32_t* seq_lens, int32_t B, void* o_gated,
                                                     void* stream) {
-  if (!cfg) {
-    gmla::set_last_error("gmla_decode_noalloc: config is NULL");
+  // the configuration and batch are checked before the scratch size is worked out
+  const gmla_status cs = static_cast<gmla_status>(gmla::check_config(cfg));
+  if (cs != GMLA_OK) return cs;
+  if (B < 0) {
+    gmla::set_last_error("gmla_decode_noalloc: B < 0");
     return GMLA_ERR_INVALID_ARG;
   }
   const size_t need = gmla_decode_workspace_size(cfg, B);

@@ -283,24 +283,28 @@ __global__ void __launch_bounds__(320, 1) prefill_attn_kernel(const __grid_const
         }
       }
       const float tmax = fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])) * a.scale_log2;
+      float alpha = 1.f;
       if (j == 0 || tmax > m + 8.f) {
         const float mn = fmaxf(m, tmax);
-        const float alpha = (m == NEG_INF) ? 0.f : ex2_approx(m - mn);
-        if (j > 0 && alpha != 1.f) {
-          // O of the previous tile is complete: S of this tile was issued after it
-#pragma unroll 1
-          for (int c = 0; c < 128; c += 16) {
-            uint32_t w[16];
-            tmem_ld16(tO + c, w);
-            tmem_ld_wait();
-#pragma unroll
-            for (int k = 0; k < 16; ++k) w[k] = __float_as_uint(__uint_as_float(w[k]) * alpha);
-            tmem_st16(tO + c, w);
-          }
-          tmem_st_wait();
-        }
+        alpha = (m == NEG_INF) ? 0.f : ex2_approx(m - mn);
         l *= alpha;
         m = mn;
+      }
+      // The raise is decided per row, but the TMEM loads and stores are
+      // warp-collective: when any row of the warp raised its max, the whole warp
+      // rescales its O rows, the others by 1. O of the previous tile is complete
+      // here: S of this tile was issued after it.
+      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll 1
+        for (int c = 0; c < 128; c += 16) {
+          uint32_t w[16];
+          tmem_ld16(tO + c, w);
+          tmem_ld_wait();
+#pragma unroll
+          for (int k = 0; k < 16; ++k) w[k] = __float_as_uint(__uint_as_float(w[k]) * alpha);
+          tmem_st16(tO + c, w);
+        }
+        tmem_st_wait();
       }
       // P over S, 32 keys at a time, the next chunk's scores read while this chunk's
       // P is computed (P of a chunk only overwrites columns already read)
@@ -330,7 +334,10 @@ __global__ void __launch_bounds__(320, 1) prefill_attn_kernel(const __grid_const
       tc_fence_before();
       mbar_arrive(&bars->p_full[x]);
     }
-    if (active && ok && mbar_wait(&bars->o_done[x], 0, abort_flag, a.status)) {
+    // warp-uniform decision: the epilogue's TMEM loads are warp-collective
+    bool epi = active && ok && mbar_wait(&bars->o_done[x], 0, abort_flag, a.status);
+    epi = __all_sync(0xffffffffu, epi);
+    if (epi) {
       tc_fence_after();
       const bool valid = qi < len;
       const int HD = a.H * kD;

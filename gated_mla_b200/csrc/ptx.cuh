@@ -213,6 +213,15 @@ __device__ __forceinline__ uint32_t cluster_ctarank() {
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
+// The two halves of a cluster barrier, executed by each thread on its own (not
+// warp-aligned): every thread of every CTA of the cluster arrives once, and a
+// wait returns when all of them have arrived.
+__device__ __forceinline__ void cluster_arrive_release() {
+  asm volatile("barrier.cluster.arrive.release;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() {
+  asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
+}
 // Address of `local` (a shared::cta address) in CTA `rank` of the cluster.
 __device__ __forceinline__ uint32_t cluster_map(uint32_t local, uint32_t rank) {
   uint32_t r;
@@ -423,16 +432,19 @@ __device__ __forceinline__ uint64_t fsub2(uint64_t a, uint64_t b) {
 
 // 2^x for two values on the FMA pipes (for x <= 2^22): x = n + f with n the
 // nearest integer (adding 1.5 * 2^23 leaves n in the low mantissa bits) and
-// |f| <= 1/2; 2^f from a degree-3 polynomial whose coefficients were fitted
-// here for relative error on [-1/2, 1/2] (at most 7.5e-5 in fp32); n is then
-// added to the exponent field. Inputs below -125 are clamped, so results
-// under 2^-125 come out as about 2^-125.
+// |f| <= 1/2; 2^f from the cubic of least maximum relative error on
+// [-1/2, 1/2], fitted by the Remez exchange algorithm with weight 2^-f
+// (gated_mla_b200/fit_exp2_poly.py prints these fp32 coefficients); evaluated
+// by fp32 Horner steps its relative error is at most 7.5e-5 (checked on a
+// dense grid by tests/test_exp2_poly.py). n is then added to the exponent
+// field, which is exact. Inputs below -125 are clamped, so results under
+// 2^-125 come out as about 2^-125.
 __device__ __forceinline__ void exp2_poly2(float x0, float x1, float& y0, float& y1) {
   const float kMagic = 12582912.f;   // 1.5 * 2^23
   const uint64_t x = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
   const uint64_t t = fadd2(x, f2_pack(kMagic, kMagic));
   const uint64_t f = fsub2(x, fsub2(t, f2_pack(kMagic, kMagic)));   // t - magic = n exactly
-  uint64_t p = ffma2(f2_pack(0.055171623826026917f, 0.055171623826026917f), f,
+  uint64_t p = ffma2(f2_pack(0.055171668529510498f, 0.055171668529510498f), f,
                      f2_pack(0.2426111251115799f, 0.2426111251115799f));
   p = ffma2(p, f, f2_pack(0.6932609677314758f, 0.6932609677314758f));
   p = ffma2(p, f, f2_pack(0.9999280571937561f, 0.9999280571937561f));

@@ -34,6 +34,8 @@
  *   - Row-major layouts. Weights are [out, in]:
  *       W_c [d_c, d_model]   W_kr [d_R, d_model]    W_q [H*d_h, d_model]
  *       W_qr [H*d_R, d_model]  W_k, W_v [H, d_h, d_c]
+ *       with a compressed query (d_cq > 0): W_dq [d_cq, d_model], W_uq [H*d_h, d_cq],
+ *       W_qr [H*d_R, d_cq], and W_q unused
  *       W_g [G, d_model] with G = H*d_h (per-channel gate) or G = H (per-head gate)
  *       b_g [G] (fp32, optional)   W_o [d_model, H*d_h]
  *     Weights, x, q, the cache, o and y use the config's dtype (bf16 or fp32);
@@ -87,6 +89,8 @@ typedef struct gmla_config {
   float softmax_scale;    /* scale applied to q.k (+ q^R.k^R) before the softmax */
   float rope_base;        /* RoPE base (e.g. 10000) */
   int32_t dtype;          /* gmla_dtype */
+  int32_t d_cq;           /* low-rank query width d_cq ("精读笔记 03" §5.1: c^Q = W^DQ h,
+                             q = W^UQ c^Q; §5.2: q^R = RoPE(W^QR c^Q)); 0 = full-rank query */
 } gmla_config;
 
 typedef struct gmla_weights {
@@ -99,6 +103,8 @@ typedef struct gmla_weights {
   const void* W_g;
   const float* b_g;       /* NULL unless gate_bias */
   const void* W_o;
+  const void* W_dq;       /* [d_cq, d_model] when d_cq > 0, else NULL */
+  const void* W_uq;       /* [H*d_h, d_cq] when d_cq > 0, else NULL */
 } gmla_weights;
 
 /* Latent cache. A row holds [c (d_c) | k^R (d_R)] of one token, d_c + d_R
@@ -126,7 +132,9 @@ typedef struct gmla_cache {
  *   seq_ids      [T] int32, sequence (cache slot) of each token
  *   cache        receives row [c | RoPE(W_kr x, pos)] of every token at (seq_id, position)
  *                ("Gated MLA 计算公式" §一; "精读笔记 03" §5.1, §5.2)
- *   q_out        [T, H, d_h + d_R]: q^(h) = W_q^(h) x, then q^R = RoPE(W_qr^(h) x, pos)
+ *   q_out        [T, H, d_h + d_R]: q^(h) = W_q^(h) x, then q^R = RoPE(W_qr^(h) x, pos);
+ *                with d_cq > 0: c^Q = W_dq x, q = W_uq c^Q, q^R = RoPE(W_qr c^Q, pos)
+ *                ("精读笔记 03" §5.1, §5.2), two GEMMs with c^Q kept in the workspace
  *   gate_logits  [T, G] fp32: W_g x (+ b_g)
  *   workspace    device scratch of gmla_latent_project_workspace_size(cfg, T) bytes
  * Rows of the cache not addressed by (seq_id, position) are left untouched.
@@ -207,13 +215,21 @@ GMLA_API gmla_status gmla_gate_out(const gmla_config* cfg, const gmla_weights* w
  *     calls whose kernels overlap on the GPU race on it, so serialise them.
  *   - Device-side faults are recorded in the shared array's status word,
  *     which each call clears first; this variant does not report them back.
+ *     A sequence length beyond the cache or a page id outside the pool
+ *     therefore gives an undefined o_gated with no error returned: callers
+ *     that cannot vouch for seq_lens and the block table should use
+ *     gmla_decode, whose workspace status gmla_sync_status() reads.
+ *   - An invalid configuration or B < 0 returns GMLA_ERR_INVALID_ARG before
+ *     anything reaches the device.
  * ------------------------------------------------------------------------- */
 GMLA_API gmla_status gmla_decode_noalloc(const gmla_config* cfg, const gmla_weights* w,
                                          const void* q, const float* gate_logits,
                                          const gmla_cache* cache, const int32_t* seq_lens,
                                          int32_t B, void* o_gated, void* stream);
 
-/* Scratch sizes in bytes (0 is never returned; 256-byte aligned). */
+/* Scratch sizes in bytes (0 is never returned; 256-byte aligned). An invalid
+ * configuration or a negative size gets 256 (the calls themselves then fail
+ * with GMLA_ERR_INVALID_ARG). */
 GMLA_API size_t gmla_latent_project_workspace_size(const gmla_config* cfg, int32_t T);
 GMLA_API size_t gmla_decode_workspace_size(const gmla_config* cfg, int32_t B);
 GMLA_API size_t gmla_prefill_workspace_size(const gmla_config* cfg, int32_t T, int32_t B);
@@ -246,6 +262,17 @@ GMLA_API gmla_status gmla_profile_enable(int32_t enable);
 GMLA_API int32_t gmla_profile_count(void);
 /* Name and duration (ms) of record i; waits for its stop event. */
 GMLA_API gmla_status gmla_profile_get(int32_t i, const char** name, float* ms);
+
+/* ---------------------------------------------------------------------------
+ * Test hook, not part of the method: arms (1) or disarms (0) a one-shot stall
+ * in the next bf16 gmla_decode on this process. In that call the tensor-core
+ * thread of the first attention block waits on a barrier that nothing
+ * completes; the wait gives up after its bound (about one second), the block
+ * leaves through its abort path, the workspace status word reads
+ * GMLA_ERR_TIMEOUT and the call's output is undefined. The device stays
+ * usable: clear the status and call again. Faults nothing, hangs nothing.
+ * ------------------------------------------------------------------------- */
+GMLA_API gmla_status gmla_test_stall_next_decode(int32_t enable);
 
 /* Library version, e.g. "gmla 0.1.0 sm_100a". */
 GMLA_API const char* gmla_version(void);

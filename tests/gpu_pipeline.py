@@ -41,11 +41,12 @@ def make_model(inp, device="cuda"):
     w = inp["workload"]
     dt = _dt(w)
     dev = lambda a, t=dt: None if a is None else torch.from_numpy(np.ascontiguousarray(a)).to(device, t)
-    weights = {k: dev(inp[k]) for k in ("W_c", "W_kr", "W_q", "W_qr", "W_k", "W_v", "W_g", "W_o")}
+    weights = {k: dev(inp.get(k)) for k in ("W_c", "W_kr", "W_q", "W_qr", "W_k", "W_v", "W_g", "W_o",
+                                            "W_dq", "W_uq")}
     weights["b_g"] = dev(inp["b_g"], torch.float32)
     return GatedMLA(d_model=w.d_model, n_heads=w.n_heads, d_h=w.d_h, d_c=w.d_c, d_rope=w.d_rope,
                     gate_mode=w.gate_mode, softmax_scale=w.softmax_scale, rope_base=w.rope_base,
-                    dtype=dt, weights=weights)
+                    dtype=dt, weights=weights, d_cq=w.d_cq)
 
 
 def make_decode_cache(inp, device="cuda", paged=None, capacity=None, fill=float("nan")):

@@ -91,3 +91,22 @@ def test_binding_names_match_the_c_abi(L):
         if s in ("gmla_status_string", "gmla_last_error", "gmla_version"):
             continue
         assert hasattr(L, s), s
+
+
+def test_bad_config_never_reaches_a_size_computation(L):
+    """n_heads = 0 (or another invalid config) must not crash a size query or
+    the no-allocation decode: the queries answer 256 and the call returns
+    GMLA_ERR_INVALID_ARG before any device work."""
+    w = L.gmla_weights()
+    k = L.gmla_cache()
+    for bad in (dict(n_heads=0), dict(d_h=-1), dict(d_c=0), dict(dtype=7)):
+        cb = _cfg(L, **bad)
+        assert L.gmla_decode_workspace_size(cb, 32) == 256, bad
+        assert L.gmla_prefill_workspace_size(cb, 64, 1) == 256, bad
+        assert L.gmla_latent_project_workspace_size(cb, 8) == 256, bad
+        assert L.gmla_gate_out_workspace_size(cb, 8) == 256, bad
+        st = L.gmla_decode_noalloc(cb, w, None, None, k, None, 4, None, None)
+        assert st == L.GMLA_ERR_INVALID_ARG, bad
+    st = L.gmla_decode_noalloc(_cfg(L), w, None, None, k, None, -1, None, None)
+    assert st == L.GMLA_ERR_INVALID_ARG
+    assert b"B < 0" in L.lib.gmla_last_error()
