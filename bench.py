@@ -2,24 +2,30 @@
 """Benchmark of the Gated MLA hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload NAME]
+                    [--workload NAME] [--prefill-workload NAME|none]
 
-Default workload: the batch-32 decode (d_model 2048, 16 heads, d_h 128,
-d_c 512, NoPE, per-channel gate, cache lengths uniform in [1024, 8192],
-seed 0). A decode step is gmla_latent_project (writes each sequence's new
-latent row) -> gmla_decode (absorbed split-K attention, W_v and gate) ->
-gmla_gate_out (W_o); its metric is latent-cache bytes read per step over the
-step time (GB/s). A prefill step (``--workload prefill_b4_s4096`` or
-``tiny_prefill_f32``) is gmla_latent_project -> gmla_prefill -> gmla_gate_out
-over whole prompts; its metric is explicit-form algorithmic FLOPs per second
-(TFLOP/s). Inputs are synthetic, drawn by ``synth``.
+One run measures two workloads on the same GPU, one after the other:
+
+* the JSON line itself: the long-context decode (batch 8 x 131072 cached rows,
+  d_model 7168, 128 heads, d_h 128, d_c 512 + decoupled RoPE 64, per-channel
+  gate, seed 0), the largest decode workload. A decode step is
+  gmla_latent_project (writes each sequence's new latent row) -> gmla_decode
+  (absorbed split-K attention, W_v and gate) -> gmla_gate_out (W_o); its metric
+  is latent-cache bytes read per step over the step time (GB/s);
+* its ``prefill`` object: the batch-4 x 4096 causal prefill (d_model 7168,
+  64 heads), a step being gmla_latent_project -> gmla_prefill -> gmla_gate_out
+  over whole prompts, with explicit-form algorithmic FLOPs per second (TFLOP/s).
+
+``--workload`` picks another decode (or prefill) workload for the line;
+``--prefill-workload none`` leaves the prefill object out. Inputs are
+synthetic, drawn by ``synth``.
 
 Timing: W untimed warm-up steps; then K steps, each replayed from a CUDA
 graph between CUDA events on the launching stream, with L2 flushed before
-every step by a 256 MiB memset and a read of it (outside the events); barrier + synchronize on
-both sides; the max over ranks of the summed step times. Under torchrun every
-rank runs its own replica of the workload (weak scaling; no data-path
-collective). Rank 0 prints one JSON line.
+every step by a 256 MiB memset and a read of it (outside the events); barrier
++ synchronize on both sides; the max over ranks of the summed step times.
+Under torchrun every rank runs its own replica of the workload (weak scaling;
+no data-path collective). Rank 0 prints one JSON line.
 
 ``--impl reference`` times the fp64 oracle (the CPU restatement of the method
 that the tests check the library against) on this machine's host cores, each
@@ -42,9 +48,13 @@ sys.path.insert(0, ROOT)
 
 DECODE_METRIC = "Gated-MLA decode latent-cache GB/s (latent_project + decode + gate_out step)"
 PREFILL_METRIC = "Gated-MLA prefill TFLOP/s (latent_project + prefill + gate_out step, explicit-form FLOPs)"
-DEFAULT_WORKLOAD = "decode_b32"
-# the pool's earlier measurement: HBM copy, bf16 GEMM burst, and the same GEMM
-# sustained under the 1 kW power cap (about 1.4 PFLOP/s near 1.3 GHz)
+DEFAULT_WORKLOAD = "decode_long_rope"
+DEFAULT_PREFILL = "prefill_b4_s4096"
+WORKLOAD_NAMES = ["decode_b32", "decode_long_rope", "decode_paged_head", "prefill_b4_s4096",
+                  "prefill_b1_s4096_h16", "tiny_prefill_f32", "decode_long_rope_qc", "prefill_b4_s4096_qc"]
+# Denominators used when no measured peaks file is present: a B200's HBM copy
+# bandwidth (GB/s), its dense bf16 GEMM throughput as a short burst, and the
+# same GEMM held for seconds under the 1 kW power cap (TFLOP/s).
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -62,9 +72,9 @@ def parse():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
-                    choices=["decode_b32", "decode_long_rope", "decode_paged_head", "prefill_b4_s4096", "prefill_b1_s4096_h16",
-                             "tiny_prefill_f32"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=WORKLOAD_NAMES)
+    ap.add_argument("--prefill-workload", default=DEFAULT_PREFILL, choices=WORKLOAD_NAMES + ["none"],
+                    help="prefill workload measured in the same run (its own object in the line)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle CPU baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
@@ -90,19 +100,38 @@ def src_hash(files):
 
 
 DECODE_SRC = ["gated_mla_b200/csrc/decode_tc.cu", "gated_mla_b200/csrc/ptx.cuh", "gated_mla_b200/csrc/common.cuh"]
+KERNEL_SRC = {
+    "decode_attn": DECODE_SRC,
+    "prefill_attn": ["gated_mla_b200/csrc/prefill_tc.cu", "gated_mla_b200/csrc/ptx.cuh",
+                     "gated_mla_b200/csrc/common.cuh"],
+    "gemm_project": ["gated_mla_b200/csrc/gemm_tc.cu", "gated_mla_b200/csrc/ptx.cuh",
+                     "gated_mla_b200/csrc/common.cuh"],
+}
 
 
-def ncu_traffic():
-    """DRAM bytes per decode_attn launch from the committed ncu summary, if it
-    was taken on the current kernel source."""
-    p = os.path.join(ROOT, "profiles", "decode_attn_decode_b32.json")
-    if not os.path.exists(p):
+def ncu_traffic(kernel, workload):
+    """DRAM bytes (read + write) per launch of `kernel` on `workload` from the
+    committed ncu summary profiles/<kernel>_<workload>.json, if it was taken on
+    the current kernel source; else None."""
+    p = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.json")
+    if not os.path.exists(p) or kernel not in KERNEL_SRC:
         return None
     with open(p) as f:
         d = json.load(f)
-    if d.get("src_sha") != src_hash(DECODE_SRC):
+    if d.get("src_sha") != src_hash(KERNEL_SRC[kernel]):
         return None
     return d.get("dram_bytes_per_launch")
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
 
 
 class ClockSampler:
@@ -170,12 +199,17 @@ def prefill_flops(w, lengths):
     """Explicit-form algorithmic FLOPs of one prefill step, per kernel."""
     T = int(sum(lengths))
     H, dh, dc, dr, dm = w.n_heads, w.d_h, w.d_c, w.d_rope, w.d_model
-    n_proj = dc + dr + H * dh + H * dr + w.gate_width
     pairs = sum(int(L) * (int(L) + 1) // 2 for L in lengths)
-    return {"gemm_project": 2.0 * T * dm * n_proj,
-            "gemm_kv": 2.0 * T * dc * 2 * H * dh,
-            "prefill_attn": 4.0 * (dh + dr) * H * pairs,
-            "gemm_out": 2.0 * T * H * dh * dm}
+    out = {}
+    if w.d_cq:   # low-rank query: x -> [c | k^R | c^Q | g], then c^Q -> [q | q^R]
+        out["gemm_project"] = 2.0 * T * dm * (dc + dr + w.d_cq + w.gate_width)
+        out["gemm_query_up"] = 2.0 * T * w.d_cq * (H * dh + H * dr)
+    else:
+        out["gemm_project"] = 2.0 * T * dm * (dc + dr + H * dh + H * dr + w.gate_width)
+    out.update({"gemm_kv": 2.0 * T * dc * 2 * H * dh,
+                "prefill_attn": 4.0 * (dh + dr) * H * pairs,
+                "gemm_out": 2.0 * T * H * dh * dm})
+    return out
 
 
 def config_dict(w, inp):
@@ -184,14 +218,17 @@ def config_dict(w, inp):
         desc = (f"{w.name}: batch {w.batch} decode, d_model {w.d_model}, H {w.n_heads}, d_h {w.d_h}, d_c {w.d_c}"
                 + (f" + RoPE {w.d_rope}" if w.d_rope else ", NoPE")
                 + (", paged (page 64)" if w.paged else "")
-                + f", {w.gate_mode} gate, lengths {w.len_law}[{w.len_lo},{w.len_hi}] seed 0")
+                + f", {w.gate_mode} gate, lengths {w.len_law}[{w.len_lo},{w.len_hi}]"
+                + (f", low-rank query d_cq {w.d_cq}" if w.d_cq else "") + ", seed 0")
         extra = {"sum_len": int(lens.sum()), "latent_bytes_per_step": int(lens.sum()) * w.row * 2}
     else:
         desc = (f"{w.name}: batch {w.batch} x {w.seq_len} causal prefill, d_model {w.d_model}, H {w.n_heads}, "
-                f"d_h {w.d_h}, d_c {w.d_c}, NoPE, {w.gate_mode} gate, {w.dtype}")
+                f"d_h {w.d_h}, d_c {w.d_c}, " + (f"RoPE {w.d_rope}" if w.d_rope else "NoPE")
+                + f", {w.gate_mode} gate" + (f", low-rank query d_cq {w.d_cq}" if w.d_cq else "")
+                + f", {w.dtype}, seed 0")
         extra = {"flops_per_step": sum(prefill_flops(w, lens).values())}
     return dict({"workload": desc, "batch": w.batch, "d_model": w.d_model, "n_heads": w.n_heads, "d_h": w.d_h,
-                 "d_c": w.d_c, "d_rope": w.d_rope,
+                 "d_c": w.d_c, "d_rope": w.d_rope, "d_cq": w.d_cq,
                  "l2": "flushed before every timed step (256 MiB memset then a read of it, outside the events)",
                  "parallelism": "replica per GPU"}, **extra)
 
@@ -266,14 +303,12 @@ def job_throughput(local_ms, world, units_per_step, steps, scale, dist=None, dev
     return world * units_per_step * steps / (max_ms / 1e3) / scale, max_ms
 
 
-def run_reference(args):
+def reference_fields(name, args, per_step):
+    """The oracle timed on a bounded sample of workload `name` per step."""
     import synth
-    if int(os.environ.get("RANK", "0")) != 0:
-        return
-    w = synth.workload(args.workload)
+    w = synth.workload(name)
     inp = synth.generate(w, seed=0)
     scale, unit = work_unit(w)
-    per_step = max(0.5, min(6.0, 150.0 / max(1, args.steps + args.warmup)))
     for i in range(args.warmup):
         oracle_sample(inp, per_step, start=i)
     tot_w, tot_s, desc = 0.0, 0.0, ""
@@ -282,17 +317,30 @@ def run_reference(args):
         tot_w += wk
         tot_s += sec
     value = tot_w / tot_s / scale
-    cores = blas_threads()
-    line = {
-        "impl": "reference", "metric": DECODE_METRIC if w.mode == "decode" else PREFILL_METRIC,
+    return {
+        "metric": DECODE_METRIC if w.mode == "decode" else PREFILL_METRIC,
         "value": value, "unit": unit, "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * tot_s / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config_dict(w, inp),
-        "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": unit, "cores": blas_threads(), "cpu_model": cpu_model(),
+                         "kind": "oracle",
                          "sample": f"per step: {desc}; fp64 explicit form (per-head K/V rebuilt from "
                                    f"latents), numpy/BLAS"},
         "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
+
+
+def run_reference(args):
+    import synth
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    with_prefill = synth.workload(args.workload).mode == "decode" and args.prefill_workload != "none"
+    per_step = max(0.5, min(6.0, 150.0 / max(1, args.steps + args.warmup)))
+    if with_prefill:
+        per_step /= 2
+    line = dict(impl="reference", **reference_fields(args.workload, args, per_step))
+    if with_prefill:
+        line["prefill"] = reference_fields(args.prefill_workload, args, per_step)
     print(json.dumps(line), flush=True)
 
 
@@ -385,23 +433,15 @@ class PrefillRunner:
         self.y_host.copy_(yy, non_blocking=True)
 
 
-def run_ours(args):
+def measure(name, args, world, rank, dev, dist, cpu_leg):
+    """Time one workload as described in the module docstring; returns the
+    fields of its JSON line (or object)."""
     import torch
-    import torch.distributed as dist
 
     import synth
     from gated_mla_b200 import _lib
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=180), device_id=dev)
-
-    w = synth.workload(args.workload)
+    w = synth.workload(name)
     inp = synth.generate(w, seed=0)
     run = DecodeRunner(inp, dev) if w.mode == "decode" else PrefillRunner(inp, dev)
     scale, unit = work_unit(w)
@@ -440,7 +480,7 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
+    with ClockSampler(dev.index) as clk:
         t_wall = time.perf_counter()
         for i in range(K):
             flush_l2(flush)
@@ -476,8 +516,8 @@ def run_ours(args):
         pgraph.replay()
         torch.cuda.synchronize()
         for i in range(n_rec):
-            name, ms = _lib.gmla_profile_get(i)
-            by.setdefault(name, []).append(ms)
+            kname, ms = _lib.gmla_profile_get(i)
+            by.setdefault(kname, []).append(ms)
     _lib.gmla_profile_enable(0)
     del pgraph
     kernel_ms = {k: statistics.mean(v) * (len(v) // K) for k, v in by.items()}   # per step
@@ -487,7 +527,7 @@ def run_ours(args):
         achieved = run.kernel_work[dom] / (kernel_ms[dom] / 1e3) / 1e9
         roof = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / pk["hbm_gbs"], "peak_source": pk["source"],
-                "traffic": ncu_traffic() if args.workload == DEFAULT_WORKLOAD else None,
+                "traffic": ncu_traffic(dom, name),
                 "launch_ms": kernel_ms[dom], "algorithmic_bytes_per_launch": run.kernel_work[dom]}
     else:
         per = {k: v for k, v in run.kernel_work.items() if k in kernel_ms}
@@ -502,8 +542,10 @@ def run_ours(args):
                 "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops_sustained"],
                 "peak_source": pk["source"] + " sustained", "peak_burst": pk["bf16_tflops"],
                 "frac_of_burst": achieved / pk["bf16_tflops"],
-                "traffic": None, "launch_ms": kernel_ms[dom], "algorithmic_flops_per_launch": per[dom],
-                "per_kernel_tflops": {k: per[k] / (kernel_ms[k] / 1e3) / 1e12 for k in per}}
+                "traffic": ncu_traffic(dom, name), "launch_ms": kernel_ms[dom],
+                "algorithmic_flops_per_launch": per[dom],
+                "per_kernel_tflops": {k: per[k] / (kernel_ms[k] / 1e3) / 1e12 for k in per},
+                "step_frac_of_sustained": value / pk["bf16_tflops_sustained"]}
 
     # end to end through the public API, host buffers (pinned), copies inside the events
     h2d = sum(t.numel() * t.element_size() for t in run.host_in)
@@ -524,27 +566,60 @@ def run_ours(args):
     run.model.sync_status()
 
     cpu = None
-    if rank == 0 and not args.no_cpu_baseline:
+    if cpu_leg:
         wk, sec, desc = oracle_sample(inp, args.cpu_seconds)
-        cpu = {"value": wk / sec / scale, "unit": unit, "cores": blas_threads(), "kind": "oracle",
+        cpu = {"value": wk / sec / scale, "unit": unit, "cores": blas_threads(), "cpu_model": cpu_model(),
+               "kind": "oracle",
                "sample": f"{desc} of the same workload, fp64 explicit form, numpy/BLAS, {sec:.1f} s"}
+    out = {
+        "metric": DECODE_METRIC if w.mode == "decode" else PREFILL_METRIC, "value": value, "unit": unit,
+        "ms_per_step": max_total_ms / K,
+        "dtype": "bf16" if w.dtype == "bf16" else "f32",
+        "config": dict(config_dict(w, inp), cuda_graph=True),
+        "roofline": roof, "kernel_ms": kernel_ms, "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": int(launches_per_step * K),
+        "clocks": clk.summary(),
+    }
+    del graph
+    del run
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=180), device_id=dev)
+
+    cpu_leg = rank == 0 and not args.no_cpu_baseline
+    main_fields = measure(args.workload, args, world, rank, dev, dist, cpu_leg)
+    pre = None
+    import synth
+    if synth.workload(args.workload).mode == "decode" and args.prefill_workload != "none":
+        pre = measure(args.prefill_workload, args, world, rank, dev, dist, cpu_leg)
     if world > 1:
         dist.barrier()
     if rank == 0:
-        line = {
-            "metric": DECODE_METRIC if w.mode == "decode" else PREFILL_METRIC, "value": value, "unit": unit,
-            "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": max_total_ms / K,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
-            "config": dict(config_dict(w, inp), cuda_graph=True),
-            "roofline": roof, "kernel_ms": kernel_ms, "cpu_baseline": cpu,
-            "e2e": {"value": e2e_value, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": int(launches_per_step * K),
-            "clocks": clk.summary(),
-        }
+        line = {"metric": main_fields.pop("metric"), "value": main_fields.pop("value"),
+                "unit": main_fields.pop("unit"), "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": main_fields.pop("ms_per_step"), "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "data": "synthetic"}
+        line.update(main_fields)
+        if pre is not None:
+            line["prefill"] = dict(pre, n_gpus=world, steps=args.steps, warmup=args.warmup,
+                                   higher_is_better=True, scaling="weak", vs_baseline=None, data="synthetic")
         print(json.dumps(line), flush=True)
     if world > 1:
-        del graph
         dist.destroy_process_group()
 
 
