@@ -51,7 +51,8 @@ PREFILL_METRIC = "Gated-MLA prefill TFLOP/s (latent_project + prefill + gate_out
 DEFAULT_WORKLOAD = "decode_long_rope"
 DEFAULT_PREFILL = "prefill_b4_s4096"
 WORKLOAD_NAMES = ["decode_b32", "decode_long_rope", "decode_paged_head", "prefill_b4_s4096",
-                  "prefill_b1_s4096_h16", "tiny_prefill_f32", "decode_long_rope_qc", "prefill_b4_s4096_qc"]
+                  "prefill_b1_s4096_h16", "tiny_prefill_f32", "decode_long_rope_qc", "prefill_b4_s4096_qc",
+                  "decode_paged_head_top8", "decode_long_rope_top32", "decode_long_rope_b2"]
 # Denominators used when no measured peaks file is present: a B200's HBM copy
 # bandwidth (GB/s), its dense bf16 GEMM throughput as a short burst, and the
 # same GEMM held for seconds under the 1 kW power cap (TFLOP/s).
@@ -219,7 +220,8 @@ def config_dict(w, inp):
                 + (f" + RoPE {w.d_rope}" if w.d_rope else ", NoPE")
                 + (", paged (page 64)" if w.paged else "")
                 + f", {w.gate_mode} gate, lengths {w.len_law}[{w.len_lo},{w.len_hi}]"
-                + (f", low-rank query d_cq {w.d_cq}" if w.d_cq else "") + ", seed 0")
+                + (f", low-rank query d_cq {w.d_cq}" if w.d_cq else "")
+                + (f", top-{w.gate_topk} of {w.n_heads} heads" if w.gate_mode == "head_topk" else "") + ", seed 0")
         extra = {"sum_len": int(lens.sum()), "latent_bytes_per_step": int(lens.sum()) * w.row * 2}
     else:
         desc = (f"{w.name}: batch {w.batch} x {w.seq_len} causal prefill, d_model {w.d_model}, H {w.n_heads}, "

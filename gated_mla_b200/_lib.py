@@ -23,6 +23,9 @@ GMLA_BF16 = 0
 GMLA_FP32 = 1
 GMLA_GATE_CHANNEL = 0
 GMLA_GATE_HEAD = 1
+GMLA_GATE_HEAD_TOPK = 2
+GMLA_GATE_HEAD_BINARY = 3
+GMLA_GATE_HEAD_TERNARY = 4
 
 
 class gmla_config(ctypes.Structure):
@@ -38,6 +41,7 @@ class gmla_config(ctypes.Structure):
         ("rope_base", ctypes.c_float),
         ("dtype", ctypes.c_int32),
         ("d_cq", ctypes.c_int32),
+        ("gate_topk", ctypes.c_int32),
     ]
 
 

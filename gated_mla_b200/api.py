@@ -15,6 +15,8 @@ import torch
 from . import _lib as L
 
 _DT = {torch.bfloat16: L.GMLA_BF16, torch.float32: L.GMLA_FP32}
+_GATE = {"channel": L.GMLA_GATE_CHANNEL, "head": L.GMLA_GATE_HEAD, "head_topk": L.GMLA_GATE_HEAD_TOPK,
+         "head_binary": L.GMLA_GATE_HEAD_BINARY, "head_ternary": L.GMLA_GATE_HEAD_TERNARY}
 
 
 def _p(t: Optional[torch.Tensor]):
@@ -59,12 +61,13 @@ class GatedMLA:
     def __init__(self, *, d_model: int, n_heads: int, d_h: int, d_c: int, d_rope: int = 0,
                  gate_mode: str = "channel", softmax_scale: Optional[float] = None,
                  rope_base: float = 10000.0, dtype: torch.dtype = torch.bfloat16,
-                 weights: dict, d_cq: int = 0):
+                 weights: dict, d_cq: int = 0, gate_topk: int = 0):
         self.dtype = dtype
         self.cfg = L.gmla_config()
         self.cfg.d_model, self.cfg.n_heads, self.cfg.d_h, self.cfg.d_c, self.cfg.d_rope = (
             d_model, n_heads, d_h, d_c, d_rope)
-        self.cfg.gate_mode = L.GMLA_GATE_CHANNEL if gate_mode == "channel" else L.GMLA_GATE_HEAD
+        self.cfg.gate_mode = _GATE[gate_mode]
+        self.cfg.gate_topk = gate_topk
         self.cfg.gate_bias = 1 if weights.get("b_g") is not None else 0
         self.cfg.softmax_scale = softmax_scale if softmax_scale else 1.0 / math.sqrt(d_h + d_rope)
         self.cfg.rope_base = rope_base

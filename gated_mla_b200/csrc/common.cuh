@@ -34,6 +34,63 @@ static __device__ __noinline__ int64_t cache_row(const CacheView& c, int b, int 
   return static_cast<int64_t>(page) * c.page_size + (pos % c.page_size);
 }
 
+// Gate modes (gmla_gate_mode): per channel, or per head as a sigmoid, hard
+// top-k, binary or ternary value.
+enum : int { kGateChannel = 0, kGateHead = 1, kGateTopk = 2, kGateBinary = 3, kGateTernary = 4 };
+
+__host__ __device__ inline bool gate_is_hard(int mode) { return mode >= kGateTopk; }
+
+// Gate value of head h of one token from its H per-head logits z
+// ("Gated Multi-head Latent Attention", "Gating Mechanism" and "Variants /
+// Extensions"): sigmoid(z_h); top-k: 1 for the k largest logits, equal logits
+// to the lower head; binary: 1 where sigmoid(z) >= 1/2, i.e. z >= 0; ternary:
+// sigmoid(z) rounded to the nearest of 0, 1/2, 1 (halves up), i.e. cut at
+// z = -ln 3 and z = ln 3.
+__device__ __forceinline__ float head_gate(const float* z, int H, int h, int mode, int k) {
+  const float zh = z[h];
+  if (mode == kGateTopk) {
+    int rank = 0;
+    for (int j = 0; j < H; ++j) {
+      const float zj = z[j];
+      rank += (zj > zh) || (zj == zh && j < h);
+    }
+    return rank < k ? 1.f : 0.f;
+  }
+  if (mode == kGateBinary) return zh >= 0.f ? 1.f : 0.f;
+  if (mode == kGateTernary) {
+    const float ln3 = 1.0986122886681098f;
+    return zh < -ln3 ? 0.f : (zh < ln3 ? 0.5f : 1.f);
+  }
+  return 1.f / (1.f + expf(-zh));
+}
+
+// Slot of head h when a token's heads are reordered so that those whose gate
+// is not 0 come first (decode computes only those). Top-k: the rank of the
+// logit; otherwise active heads by index, then the others by index. *n_act
+// gets the number of active heads.
+__device__ __forceinline__ int head_slot(const float* z, int H, int h, int mode, int k, int* n_act) {
+  if (mode == kGateTopk) {
+    int rank = 0;
+    for (int j = 0; j < H; ++j) {
+      const float zj = z[j], zh = z[h];
+      rank += (zj > zh) || (zj == zh && j < h);
+    }
+    *n_act = k;
+    return rank;
+  }
+  int act = 0, before_act = 0, before_off = 0;
+  for (int j = 0; j < H; ++j) {
+    const bool on = head_gate(z, H, j, mode, k) != 0.f;
+    act += on;
+    if (j < h) {
+      before_act += on;
+      before_off += !on;
+    }
+  }
+  *n_act = act;
+  return head_gate(z, H, h, mode, k) != 0.f ? before_act : act + before_off;
+}
+
 // How a GEMM epilogue writes one weight segment's outputs.
 // Element (token t, feature f) goes to
 //   out + row(t) * row_stride + (f / block) * block_stride + (f % block) + col_offset
@@ -50,10 +107,12 @@ struct EpiSeg {
   int32_t out_f32;       // 1: fp32 output, 0: bf16 output
   int32_t rope;
   int32_t cache_scatter;
-  // optional sigmoid gate: v *= sigmoid(gate[t * gate_stride + f / gate_div])
+  // optional gate: v *= sigmoid(gate[t * gate_stride + f / gate_div]), or with
+  // gate_value set v *= gate[...] (gate values computed beforehand)
   const float* gate;
   int32_t gate_stride;
   int32_t gate_div;
+  int32_t gate_value;
 };
 
 constexpr int kMaxSeg = 5;
@@ -105,7 +164,10 @@ static __device__ __noinline__ float rope_rotate(float v, float partner, bool od
 }
 
 __device__ __forceinline__ void epi_store(const EpiSeg& e, int64_t row, int f, float v, int t = 0) {
-  if (e.gate) v *= __fdividef(1.f, 1.f + __expf(-e.gate[static_cast<int64_t>(t) * e.gate_stride + f / e.gate_div]));
+  if (e.gate) {
+    const float g = e.gate[static_cast<int64_t>(t) * e.gate_stride + f / e.gate_div];
+    v *= e.gate_value ? g : __fdividef(1.f, 1.f + __expf(-g));
+  }
   const int64_t off = row * e.row_stride + static_cast<int64_t>(f / e.block) * e.block_stride + (f % e.block) +
                       e.col_offset;
   if (e.bias) v += e.bias[f];

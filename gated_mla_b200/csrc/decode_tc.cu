@@ -121,6 +121,13 @@ __device__ void decode_plan_block(const DecodeArgs& a) {
   if (tid == 0) a.seq_first_seg[a.B] = seg_carry;
   const int g_used = total > 0 ? (total - 1) / tpc + 1 : 0;
   for (int g = g_used + tid; g <= a.G; g += blockDim.x) a.cta_first_seg[g] = seg_carry;
+  if (a.gate_hard) {   // heads of each sequence whose gate is not 0
+    for (int b = tid; b < a.B; b += blockDim.x) {
+      int na = 0;
+      head_slot(a.gate_logits + static_cast<int64_t>(b) * a.H, a.H, 0, a.gate_mode, a.gate_topk, &na);
+      a.n_act[b] = na;
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -169,6 +176,28 @@ __global__ void __launch_bounds__(256, 4) decode_absorb_plan_kernel(DecodeArgs a
   };
   load_w(k_lo);
   griddep_wait();
+  // with hard / quantised gates each sequence stores its heads by slot (heads
+  // whose gate is 0 last, their rows zero); otherwise slot = head
+  __shared__ int s_slot[kAbsorbB];
+  __shared__ float s_on[kAbsorbB];
+  if (threadIdx.x < kAbsorbB) {
+    int slot = h;
+    float on = 1.f;
+    const int bi = threadIdx.x;
+    if (a.gate_hard && bi < nb) {
+      const float* z = a.gate_logits + static_cast<int64_t>(b0 + bi) * a.H;
+      int na = 0;
+      slot = head_slot(z, a.H, h, a.gate_mode, a.gate_topk, &na);
+      const float gv = head_gate(z, a.H, h, a.gate_mode, a.gate_topk);
+      on = gv != 0.f ? 1.f : 0.f;
+      if (cb == 0) {
+        a.gvals[static_cast<int64_t>(b0 + bi) * a.H + h] = gv;
+        a.head_of_slot[static_cast<int64_t>(b0 + bi) * a.H + slot] = h;
+      }
+    }
+    s_slot[bi] = slot;
+    s_on[bi] = on;
+  }
   const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(a.q);
   for (int i = threadIdx.x; i < kAbsorbB * a.d_h; i += blockDim.x) {
     const int bi = i / a.d_h, k = i % a.d_h;
@@ -208,15 +237,16 @@ __global__ void __launch_bounds__(256, 4) decode_absorb_plan_kernel(DecodeArgs a
     float v = 0.f;
 #pragma unroll
     for (int g = 0; g < kAbsorbKG; ++g) v += red[g][bi][c];
-    qa[(static_cast<int64_t>(b0 + bi) * a.H + h) * row + cb * kAbsorbCols + c] = __float2bfloat16_rn(v * a.q_scale);
+    qa[(static_cast<int64_t>(b0 + bi) * a.H + s_slot[bi]) * row + cb * kAbsorbCols + c] =
+        __float2bfloat16_rn(v * a.q_scale * s_on[bi]);
   }
   // decoupled RoPE query dims: copied (already rotated), scaled
   if (cb == 0) {
     for (int i = threadIdx.x; i < nb * a.d_rope; i += blockDim.x) {
       const int bi = i / a.d_rope, r = i % a.d_rope;
       const int64_t src = (static_cast<int64_t>(b0 + bi) * a.H + h) * dq + a.d_h + r;
-      qa[(static_cast<int64_t>(b0 + bi) * a.H + h) * row + a.d_c + r] =
-          __float2bfloat16_rn(__bfloat162float(q[src]) * a.q_scale);
+      qa[(static_cast<int64_t>(b0 + bi) * a.H + s_slot[bi]) * row + a.d_c + r] =
+          __float2bfloat16_rn(__bfloat162float(q[src]) * a.q_scale * s_on[bi]);
     }
   }
 }
@@ -259,6 +289,15 @@ struct DecCfg {
   static constexpr int kTmemCols = (6 * HG <= 128) ? 128 : ((6 * HG <= 256) ? 256 : 512);
   static_assert(kRing >= kNcBox, "ring must hold one tile");
 };
+
+// Heads of head group hg that sequence b attends with: all of the group's heads,
+// or with hard / quantised gates those whose slot is below the sequence's count
+// of active heads (0: the segment is skipped by every role of the block).
+__device__ __forceinline__ int seg_heads(const DecodeArgs& a, int b, int hg, int heads_valid) {
+  if (!a.gate_hard) return heads_valid;
+  const int n = a.n_act[b] - hg * a.HG;
+  return n <= 0 ? 0 : (n < heads_valid ? n : heads_valid);
+}
 
 template <int HG, int NBOX>
 __global__ void __launch_bounds__(64 + 128 * (HG >= 32 ? 2 : 1), 1) decode_attn_kernel(const __grid_constant__ DecodeArgs a) {
@@ -331,6 +370,7 @@ __global__ void __launch_bounds__(64 + 128 * (HG >= 32 ? 2 : 1), 1) decode_attn_
       const int4 sg = a.seg_info[si];
       const int b = sg.x;
       const int L = a.seq_lens[b];
+      if (seg_heads(a, b, hg, heads_valid) == 0) continue;
       if (lane == 0) {
         if (nq > 0 && !mbar_wait(&sm->q_empty, (nq - 1) & 1, abort_flag, a.status)) ok = false;
         if (ok) {
@@ -423,8 +463,9 @@ __global__ void __launch_bounds__(64 + 128 * (HG >= 32 ? 2 : 1), 1) decode_attn_
                       (p | b2 | kk) != 0);
         }
       };
-      for (int si = seg_lo; si < seg_hi && ok; ++si, ++nseg) {
+      for (int si = seg_lo; si < seg_hi && ok; ++si) {
         const int4 sg = a.seg_info[si];
+        if (seg_heads(a, sg.x, hg, heads_valid) == 0) continue;
         if (!mbar_wait(&sm->q_full, nseg & 1, abort_flag, a.status)) { ok = false; break; }
         for (int t = sg.y; t < sg.z; ++t, ++ntile) {
           const uint32_t tSb = tmem + (ntile & 1) * HG;
@@ -476,6 +517,7 @@ __global__ void __launch_bounds__(64 + 128 * (HG >= 32 ? 2 : 1), 1) decode_attn_
         }
         if (!ok) break;
         umma_commit(&sm->o_done);
+        ++nseg;
       }
       if (!ok) {
         umma_commit(&sm->drain);
@@ -498,9 +540,11 @@ __global__ void __launch_bounds__(64 + 128 * (HG >= 32 ? 2 : 1), 1) decode_attn_
     // the same sequence of barriers and the block can exit.
     uint32_t nbox = 0, ntile = 0, nseg = 0;
     bool ok = true;
-    for (int si = seg_lo; si < seg_hi; ++si, ++nseg) {
+    for (int si = seg_lo; si < seg_hi; ++si) {
       const int4 sg = a.seg_info[si];
       const int L = a.seq_lens[sg.x];
+      const int hv = seg_heads(a, sg.x, hg, heads_valid);
+      if (hv == 0) continue;
       float m[HT], lsum[HT];
 #pragma unroll
       for (int h = 0; h < HT; ++h) {
@@ -637,7 +681,7 @@ __global__ void __launch_bounds__(64 + 128 * (HG >= 32 ? 2 : 1), 1) decode_attn_
       }
       asm volatile("bar.sync 1, %0;" ::"n"(128 * SG) : "memory");
       const int64_t pbase = (static_cast<int64_t>(hg) * a.max_seg + si) * HG;
-      if (ok && ltid < heads_valid) {
+      if (ok && ltid < hv) {
         float l = 0.f, mh = NEG_INF;
         if (SG == 1) {   // every thread holds the running max of every head
 #pragma unroll
@@ -659,7 +703,7 @@ __global__ void __launch_bounds__(64 + 128 * (HG >= 32 ? 2 : 1), 1) decode_attn_
           tmem_ld_wait();
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            if (ok && h0 + c + j < heads_valid)
+            if (ok && h0 + c + j < hv)
               a.o_part[(pbase + h0 + c + j) * kDc + mc * 128 + row] = __uint_as_float(v[j]);
           }
         }
@@ -667,6 +711,7 @@ __global__ void __launch_bounds__(64 + 128 * (HG >= 32 ? 2 : 1), 1) decode_attn_
       tc_fence_before();
       asm volatile("bar.sync 1, %0;" ::"n"(128 * SG) : "memory");   // lred / mfin reuse
       mbar_arrive(&sm->o_free);
+      ++nseg;
     }
   }
 
@@ -690,10 +735,20 @@ __global__ void __launch_bounds__(64 + 128 * (HG >= 32 ? 2 : 1), 1) decode_attn_
 __global__ void __launch_bounds__(128) decode_merge_kernel(DecodeArgs a) {
   if (threadIdx.x == 0) griddep_launch_dependents();
   griddep_wait();
-  const int h = blockIdx.x, b = blockIdx.y;
-  const int hg = h / a.HG, hl = h % a.HG;
-  if (h == 0 && b == 0)
+  const int slot = blockIdx.x, b = blockIdx.y;
+  const int hg = slot / a.HG, hl = slot % a.HG;
+  if (slot == 0 && b == 0)
     for (int i = threadIdx.x; i < a.n_gemm_tiles; i += blockDim.x) a.gemm_counters[i] = 0;
+  int h = slot;
+  if (a.gate_hard) {
+    // slot -> head; a head whose gate is 0 was skipped: its latent output is 0
+    h = a.head_of_slot[static_cast<int64_t>(b) * a.H + slot];
+    if (slot >= a.n_act[b]) {
+      __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.olat) + (static_cast<int64_t>(h) * a.B + b) * kDc;
+      for (int j = threadIdx.x; j < kDc; j += blockDim.x) dst[j] = __float2bfloat16_rn(0.f);
+      return;
+    }
+  }
   const int s0 = a.seq_first_seg[b], s1 = a.seq_first_seg[b + 1];
   const int64_t base = static_cast<int64_t>(hg) * a.max_seg;
   // one pass over the segments, rescaling the running sums when the max grows
@@ -728,10 +783,11 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(DecodeArgs a) {
 // ---------------------------------------------------------------------------
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-DecodeLayout decode_layout(int B, int H, int d_h, int d_c, int d_rope, int num_sms) {
+DecodeLayout decode_layout(int B, int H, int eff_heads, int d_h, int d_c, int d_rope, int num_sms) {
   DecodeLayout L{};
-  L.HG = H <= 16 ? 16 : (H % 64 == 0 ? 64 : (H % 32 == 0 ? 32 : 16));
-  L.n_hg = (H + L.HG - 1) / L.HG;
+  const int E = eff_heads;
+  L.HG = E <= 16 ? 16 : (E % 64 == 0 ? 64 : (E % 32 == 0 ? 32 : 16));
+  L.n_hg = (E + L.HG - 1) / L.HG;
   L.G = num_sms / L.n_hg;
   if (L.G < 1) L.G = 1;
   L.max_seg = L.G + B + 1;
@@ -754,6 +810,12 @@ DecodeLayout decode_layout(int B, int H, int d_h, int d_c, int d_rope, int num_s
   L.off_gemm = off;
   L.gemm_plan = gemm_swap_plan(H * d_h / 128, B, d_c, num_sms);
   off = align256(off + L.gemm_plan.ws_bytes);
+  L.off_gvals = off;
+  off = align256(off + static_cast<size_t>(B) * H * 4);
+  L.off_hslot = off;
+  off = align256(off + static_cast<size_t>(B) * H * 4);
+  L.off_nact = off;
+  off = align256(off + static_cast<size_t>(B) * 4);
   L.total = off;
   return L;
 }

@@ -303,7 +303,7 @@ __global__ void __launch_bounds__(192, kSwap ? 1 : 2) gemm_bf16_tc_kernel(const 
             const int64_t row = tok_row[tl];
             if (row < 0 || !f_ok) continue;
             val += fbias;
-            if (e.gate) val *= __fdividef(1.f, 1.f + __expf(-gl[j]));
+            if (e.gate) val *= e.gate_value ? gl[j] : __fdividef(1.f, 1.f + __expf(-gl[j]));
             const int64_t off = row * e.row_stride + colpart;
             if (e.out_f32)
               static_cast<float*>(e.out)[off] = val;
@@ -489,7 +489,7 @@ __global__ void __launch_bounds__(192, kSwap ? 1 : 2) gemm_bf16_tc_kernel(const 
             const int64_t row = tok_row[tl];
             if (row < 0 || !f_ok || !got) continue;
             val += fbias;
-            if (e.gate) val *= __fdividef(1.f, 1.f + __expf(-gl[j]));
+            if (e.gate) val *= e.gate_value ? gl[j] : __fdividef(1.f, 1.f + __expf(-gl[j]));
             const int64_t off = row * e.row_stride + colpart;
             if (e.out_f32)
               static_cast<float*>(e.out)[off] = val;

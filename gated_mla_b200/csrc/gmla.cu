@@ -88,8 +88,10 @@ gmla_status check_cfg(const gmla_config* c) {
   if (c->d_model <= 0 || c->n_heads <= 0 || c->d_h <= 0 || c->d_c <= 0 || c->d_rope < 0 || c->d_cq < 0)
     return fail(GMLA_ERR_INVALID_ARG, "non-positive dimension in config");
   if (c->d_rope % 2) return fail(GMLA_ERR_INVALID_ARG, "d_rope must be even (RoPE rotates pairs)");
-  if (c->gate_mode != GMLA_GATE_CHANNEL && c->gate_mode != GMLA_GATE_HEAD)
-    return fail(GMLA_ERR_INVALID_ARG, "gate_mode must be GMLA_GATE_CHANNEL or GMLA_GATE_HEAD");
+  if (c->gate_mode < GMLA_GATE_CHANNEL || c->gate_mode > GMLA_GATE_HEAD_TERNARY)
+    return fail(GMLA_ERR_INVALID_ARG, "gate_mode must be one of the gmla_gate_mode values");
+  if (c->gate_mode == GMLA_GATE_HEAD_TOPK && (c->gate_topk < 1 || c->gate_topk > c->n_heads))
+    return fail(GMLA_ERR_INVALID_ARG, "gate_topk must be in [1, n_heads] for GMLA_GATE_HEAD_TOPK");
   if (c->dtype != GMLA_BF16 && c->dtype != GMLA_FP32) return fail(GMLA_ERR_INVALID_ARG, "dtype");
   if (!(c->softmax_scale > 0.f) || !std::isfinite(c->softmax_scale))
     return fail(GMLA_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
@@ -104,7 +106,8 @@ bool cfg_valid(const gmla_config* c) {
   if (c->d_model <= 0 || c->n_heads <= 0 || c->d_h <= 0 || c->d_c <= 0 || c->d_rope < 0 || c->d_cq < 0)
     return false;
   if (c->d_rope % 2) return false;
-  if (c->gate_mode != GMLA_GATE_CHANNEL && c->gate_mode != GMLA_GATE_HEAD) return false;
+  if (c->gate_mode < GMLA_GATE_CHANNEL || c->gate_mode > GMLA_GATE_HEAD_TERNARY) return false;
+  if (c->gate_mode == GMLA_GATE_HEAD_TOPK && (c->gate_topk < 1 || c->gate_topk > c->n_heads)) return false;
   if (c->dtype != GMLA_BF16 && c->dtype != GMLA_FP32) return false;
   if (!(c->softmax_scale > 0.f) || !std::isfinite(c->softmax_scale)) return false;
   if (c->d_rope && !(c->rope_base > 1.f)) return false;
@@ -157,6 +160,12 @@ CacheView cache_view(const gmla_config* c, const gmla_cache* k) {
 
 int gate_width(const gmla_config* c) {
   return c->gate_mode == GMLA_GATE_CHANNEL ? c->n_heads * c->d_h : c->n_heads;
+}
+
+// Most heads one decode query attends with: k under top-k gates (the others
+// are skipped), else H. The attention kernel's head groups cover this many.
+int decode_eff_heads(const gmla_config* c) {
+  return c->gate_mode == GMLA_GATE_HEAD_TOPK ? c->gate_topk : c->n_heads;
 }
 
 EpiSeg plain_seg(void* out, int64_t row_stride, int block, int block_stride, int col_offset, bool f32,
@@ -313,7 +322,7 @@ size_t gmla_gate_out_workspace_size(const gmla_config* cfg, int32_t T) {
 size_t gmla_decode_workspace_size(const gmla_config* cfg, int32_t B) {
   if (!cfg_valid(cfg) || B < 0) return 256;
   if (cfg->dtype == GMLA_FP32) return 256;
-  return decode_layout(B, cfg->n_heads, cfg->d_h, cfg->d_c, cfg->d_rope, num_sms()).total;
+  return decode_layout(B, cfg->n_heads, decode_eff_heads(cfg), cfg->d_h, cfg->d_c, cfg->d_rope, num_sms()).total;
 }
 
 size_t gmla_prefill_workspace_size(const gmla_config* cfg, int32_t T, int32_t B) {
@@ -528,6 +537,7 @@ gmla_status gmla_decode(const gmla_config* cfg, const gmla_weights* w, const voi
     a.d_c = cfg->d_c;
     a.d_rope = cfg->d_rope;
     a.gate_mode = cfg->gate_mode;
+    a.gate_topk = cfg->gate_topk;
     a.scale = cfg->softmax_scale;
     a.status = status;
     cudaError_t e = launch_attn_f32(a, st);
@@ -537,7 +547,8 @@ gmla_status gmla_decode(const gmla_config* cfg, const gmla_weights* w, const voi
   if (cfg->d_c != 512 || (cfg->d_rope != 0 && cfg->d_rope != 64))
     return fail(GMLA_ERR_UNSUPPORTED, "bf16 decode covers d_c = 512 with d_rope in {0, 64}");
   if (cfg->d_h != 128 && cfg->d_h != 256) return fail(GMLA_ERR_UNSUPPORTED, "bf16 decode covers d_h in {128, 256}");
-  const DecodeLayout L = decode_layout(B, cfg->n_heads, cfg->d_h, cfg->d_c, cfg->d_rope, num_sms());
+  const DecodeLayout L = decode_layout(B, cfg->n_heads, decode_eff_heads(cfg), cfg->d_h, cfg->d_c, cfg->d_rope,
+                                       num_sms());
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   DecodeArgs a{};
   const int row = cfg->d_c + cfg->d_rope;
@@ -581,6 +592,11 @@ gmla_status gmla_decode(const gmla_config* cfg, const gmla_weights* w, const voi
   a.max_seg = L.max_seg;
   a.q_scale = cfg->softmax_scale * 1.4426950408889634f;
   a.test_stall = g_test_stall.exchange(0);
+  a.gate_hard = (gate_is_hard(cfg->gate_mode) && gate_logits) ? 1 : 0;
+  a.gate_topk = cfg->gate_topk;
+  a.gvals = reinterpret_cast<float*>(ws + L.off_gvals);
+  a.head_of_slot = reinterpret_cast<int32_t*>(ws + L.off_hslot);
+  a.n_act = reinterpret_cast<int32_t*>(ws + L.off_nact);
   a.olat = ws + L.off_olat;
   const SwapPlan& sp = L.gemm_plan;
   a.gemm_counters = nullptr;
@@ -595,7 +611,9 @@ gmla_status gmla_decode(const gmla_config* cfg, const gmla_weights* w, const voi
       !make_tmap_2d(&g.wt[0], w->W_v, cfg->d_c, HD, static_cast<uint64_t>(cfg->d_c) * 2, 64, 128, true))
     return fail(GMLA_ERR_CUDA, "tensor maps for the W_v product failed");
   g.epi[0] = plain_seg(o_gated, HD, 1 << 30, 0, 0, false, nullptr, false, false);
-  g.epi[0].gate = gate_logits;
+  // hard / quantised gates: the values the absorb kernel computed, else sigmoid of the logits
+  g.epi[0].gate = a.gate_hard ? a.gvals : gate_logits;
+  g.epi[0].gate_value = a.gate_hard;
   g.epi[0].gate_stride = G;
   g.epi[0].gate_div = cfg->gate_mode == GMLA_GATE_CHANNEL ? 1 : cfg->d_h;
   g.seg_rows[0] = HD;
@@ -661,6 +679,7 @@ gmla_status gmla_prefill(const gmla_config* cfg, const gmla_weights* w, const vo
     a.d_c = cfg->d_c;
     a.d_rope = cfg->d_rope;
     a.gate_mode = cfg->gate_mode;
+    a.gate_topk = cfg->gate_topk;
     a.max_len = max_seqlen;
     a.scale = cfg->softmax_scale;
     a.status = status;
@@ -720,6 +739,7 @@ gmla_status gmla_prefill(const gmla_config* cfg, const gmla_weights* w, const vo
   p.H = H;
   p.d_h = cfg->d_h;
   p.gate_mode = cfg->gate_mode;
+  p.gate_topk = cfg->gate_topk;
   p.q_tiles_per_seq = tps;
   p.scale_log2 = cfg->softmax_scale * 1.4426950408889634f;
   e = launch_prefill_attn_bf16(p, st);
@@ -749,7 +769,8 @@ gmla_status gmla_gate_out(const gmla_config* cfg, const gmla_weights* w, const v
   const void* src = o;
   if (gate_logits) {
     void* tmp = static_cast<uint8_t*>(workspace) + 256;
-    cudaError_t e = launch_gate_apply(o, gate_logits, tmp, T, cfg->n_heads, cfg->d_h, cfg->gate_mode, f32, st);
+    cudaError_t e = launch_gate_apply(o, gate_logits, tmp, T, cfg->n_heads, cfg->d_h, cfg->gate_mode, cfg->gate_topk,
+                                      f32, st);
     if (e != cudaSuccess) return cuda_fail(e, "gate_out: gate");
     src = tmp;
   }

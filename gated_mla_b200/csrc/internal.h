@@ -82,14 +82,25 @@ struct DecodeArgs {
   int32_t HG, n_hg, G, max_seg;
   float q_scale;             // softmax_scale * log2(e), folded into the absorbed query
   int32_t test_stall;        // test hook: the first CTA's MMA thread waits on a barrier nothing completes
+  // hard / quantised per-head gates: heads whose gate is 0 are skipped. The
+  // absorbed queries of sequence b are stored by slot (active heads first);
+  // head_of_slot maps a slot back to its head.
+  int32_t gate_hard;         // 1: gate_mode is top-k, binary or ternary and gate logits are given
+  int32_t gate_topk;
+  float* gvals;              // workspace: [B, H] gate values
+  int32_t* head_of_slot;     // workspace: [B, H]
+  int32_t* n_act;            // workspace: [B] heads whose gate is not 0
 };
 
 struct DecodeLayout {
-  size_t off_qa, off_opart, off_ml, off_seg, off_seqfirst, off_ctafirst, off_olat, off_gemm, total;
+  size_t off_qa, off_opart, off_ml, off_seg, off_seqfirst, off_ctafirst, off_olat, off_gemm;
+  size_t off_gvals, off_hslot, off_nact, total;
   int HG, n_hg, G, max_seg;
   SwapPlan gemm_plan;        // the W_v GEMM (heads x 128 rows, B tokens, K = d_c)
 };
-DecodeLayout decode_layout(int B, int H, int d_h, int d_c, int d_rope, int num_sms);
+// eff_heads: the most heads a sequence attends with (H, or k with top-k gates),
+// which sets the head groups of the attention kernel.
+DecodeLayout decode_layout(int B, int H, int eff_heads, int d_h, int d_c, int d_rope, int num_sms);
 cudaError_t launch_decode_bf16(DecodeArgs& a, cudaStream_t st);
 
 // ----- fp32 CUDA-core path (simt_f32.cu) -----
@@ -119,7 +130,7 @@ struct AttnF32Args {
   float* o;
   const int32_t* cu_seqlens; // prefill: [B+1]; null for decode
   const int32_t* seq_lens;   // decode: [B]
-  int32_t B, T, H, d_h, d_c, d_rope, gate_mode, max_len;
+  int32_t B, T, H, d_h, d_c, d_rope, gate_mode, gate_topk, max_len;
   float scale;
   float* scratch;            // [B*H*(d_c + max_len)] or per-launch scratch
   int* status;
@@ -135,14 +146,14 @@ struct PrefillArgs {
   void* o;                   // [T, H*d_h]
   const int32_t* cu_seqlens;
   int* status;
-  int32_t B, T, H, d_h, gate_mode, q_tiles_per_seq;
+  int32_t B, T, H, d_h, gate_mode, gate_topk, q_tiles_per_seq;
   float scale_log2;
 };
 cudaError_t launch_prefill_attn_bf16(const PrefillArgs& a, cudaStream_t st);
 
 // ----- elementwise helpers (gmla.cu) -----
 cudaError_t launch_gate_apply(const void* o, const float* g, void* out, int T, int H, int d_h, int gate_mode,
-                              int is_f32, cudaStream_t st);
+                              int gate_topk, int is_f32, cudaStream_t st);
 
 // ----- error message of the current host thread (gmla.cu) -----
 void set_last_error(const char* msg);

@@ -345,7 +345,9 @@ __global__ void __launch_bounds__(320, 1) prefill_attn_kernel(const __grid_const
       const int64_t tok = beg + qi;
       const float inv = 1.f / l;
       float gh = 1.f;
-      if (valid && a.gate_logits && a.gate_mode != 0) gh = __fdividef(1.f, 1.f + __expf(-__ldg(a.gate_logits + tok * G + h)));
+      if (valid && a.gate_logits && a.gate_mode != 0)
+        gh = gate_is_hard(a.gate_mode) ? head_gate(a.gate_logits + tok * G, a.H, h, a.gate_mode, a.gate_topk)
+                                       : __fdividef(1.f, 1.f + __expf(-__ldg(a.gate_logits + tok * G + h)));
 #pragma unroll 1
       for (int c = 0; c < 128; c += 32) {
         // the gate logits first, so their latency overlaps the TMEM read

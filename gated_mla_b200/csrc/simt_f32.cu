@@ -145,6 +145,15 @@ __global__ void __launch_bounds__(kAttnThreads) attn_f32_kernel(const AttnF32Arg
     for (int i = threadIdx.x; i < a.d_h; i += blockDim.x) out[i] = 0.f;
     return;
   }
+  // per-head gates are one value per (token, head); a head whose gate is 0 is skipped
+  float gh = 1.f;
+  if (a.gate_logits && a.gate_mode != 0) {
+    gh = head_gate(a.gate_logits + static_cast<int64_t>(qi) * G, a.H, h, a.gate_mode, a.gate_topk);
+    if (gh == 0.f) {
+      for (int i = threadIdx.x; i < a.d_h; i += blockDim.x) out[i] = 0.f;
+      return;
+    }
+  }
   const float* q = a.q + (static_cast<int64_t>(qi) * a.H + h) * dq;
   for (int i = threadIdx.x; i < dq; i += blockDim.x) sq[i] = q[i];
   __syncthreads();
@@ -208,8 +217,12 @@ __global__ void __launch_bounds__(kAttnThreads) attn_f32_kernel(const AttnF32Arg
     float v = 0.f;
     for (int d = 0; d < a.d_c; ++d) v = fmaf(Wv[static_cast<int64_t>(i) * a.d_c + d], sqlat[d], v);
     if (a.gate_logits) {
-      const float zg = a.gate_logits[static_cast<int64_t>(qi) * G + (a.gate_mode == 0 ? h * a.d_h + i : h)];
-      v *= 1.f / (1.f + expf(-zg));
+      if (a.gate_mode == 0) {
+        const float zg = a.gate_logits[static_cast<int64_t>(qi) * G + h * a.d_h + i];
+        v *= 1.f / (1.f + expf(-zg));
+      } else {
+        v *= gh;
+      }
     }
     out[i] = v;
   }
@@ -228,14 +241,10 @@ cudaError_t launch_attn_f32(const AttnF32Args& a, cudaStream_t st) {
 // out = sigmoid(g) ⊙ o  (per channel, or per head broadcast over d_h)
 // ---------------------------------------------------------------------------
 __global__ void gate_apply_kernel(const void* o, const float* g, void* out, int64_t n, int HD, int H, int d_h,
-                                  int gate_mode, int is_f32) {
-  const int G = gate_mode == 0 ? HD : H;
+                                  int is_f32) {
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t t = i / HD;
-    const int c = static_cast<int>(i % HD);
-    const float z = g[t * G + (gate_mode == 0 ? c : c / d_h)];
-    const float s = 1.f / (1.f + expf(-z));
+    const float s = 1.f / (1.f + expf(-g[i]));   // per channel: G = HD, same index as o
     if (is_f32) {
       static_cast<float*>(out)[i] = static_cast<const float*>(o)[i] * s;
     } else {
@@ -245,15 +254,44 @@ __global__ void gate_apply_kernel(const void* o, const float* g, void* out, int6
   }
 }
 
+// per-head gates (sigmoid, top-k, binary, ternary): one warp per (token, head),
+// the gate value computed once from the token's H logits, lanes over d_h
+__global__ void gate_apply_head_kernel(const void* o, const float* g, void* out, int T, int H, int d_h,
+                                       int gate_mode, int gate_topk, int is_f32) {
+  const int lane = threadIdx.x & 31;
+  const int64_t pairs = static_cast<int64_t>(T) * H;
+  for (int64_t p = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5; p < pairs;
+       p += (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5) {
+    const int64_t t = p / H;
+    const int h = static_cast<int>(p % H);
+    const float s = head_gate(g + t * H, H, h, gate_mode, gate_topk);
+    const int64_t base = p * d_h;
+    for (int c = lane; c < d_h; c += 32) {
+      if (is_f32) {
+        static_cast<float*>(out)[base + c] = static_cast<const float*>(o)[base + c] * s;
+      } else {
+        const float v = __bfloat162float(static_cast<const __nv_bfloat16*>(o)[base + c]);
+        static_cast<__nv_bfloat16*>(out)[base + c] = __float2bfloat16_rn(v * s);
+      }
+    }
+  }
+}
+
 cudaError_t launch_gate_apply(const void* o, const float* g, void* out, int T, int H, int d_h, int gate_mode,
-                              int is_f32, cudaStream_t st) {
+                              int gate_topk, int is_f32, cudaStream_t st) {
   const int64_t n = static_cast<int64_t>(T) * H * d_h;
   if (n == 0) return cudaSuccess;
   const int threads = 256;
-  const int64_t blocks = (n + threads - 1) / threads;
   prof_begin(st, "gate_apply");
-  gate_apply_kernel<<<static_cast<int>(blocks < 4096 ? blocks : 4096), threads, 0, st>>>(o, g, out, n, H * d_h, H,
-                                                                                           d_h, gate_mode, is_f32);
+  if (gate_mode == 0) {
+    const int64_t blocks = (n + threads - 1) / threads;
+    gate_apply_kernel<<<static_cast<int>(blocks < 4096 ? blocks : 4096), threads, 0, st>>>(o, g, out, n, H * d_h,
+                                                                                             H, d_h, is_f32);
+  } else {
+    const int64_t blocks = (static_cast<int64_t>(T) * H * 32 + threads - 1) / threads;
+    gate_apply_head_kernel<<<static_cast<int>(blocks < 4096 ? blocks : 4096), threads, 0, st>>>(
+        o, g, out, T, H, d_h, gate_mode, gate_topk, is_f32);
+  }
   prof_end(st);
   return cudaGetLastError();
 }

@@ -75,8 +75,23 @@ typedef enum gmla_dtype { GMLA_BF16 = 0, GMLA_FP32 = 1 } gmla_dtype;
 
 /* Per-channel gate: G = H*d_h ("Gated MLA 计算公式" §二 boxed equation).
  * Per-head gate:    G = H, broadcast over the head's d_h channels
- *                   ("Gated Multi-head Latent Attention", "Gating Mechanism"). */
-typedef enum gmla_gate_mode { GMLA_GATE_CHANNEL = 0, GMLA_GATE_HEAD = 1 } gmla_gate_mode;
+ *                   ("Gated Multi-head Latent Attention", "Gating Mechanism").
+ * Per-head hard and quantised gates ("Gated Multi-head Latent Attention",
+ * "Variants / Extensions": Hard Gating, Quantized Gates), also G = H:
+ *   GMLA_GATE_HEAD_TOPK     1 for the gate_topk heads with the largest logits of
+ *                           the token (equal logits: lower head first), else 0
+ *   GMLA_GATE_HEAD_BINARY   1 where sigmoid(z) >= 1/2 (z >= 0), else 0
+ *   GMLA_GATE_HEAD_TERNARY  sigmoid(z) rounded to the nearest of 0, 1/2, 1
+ *                           (halves up): 0 below z = -ln 3, 1 from z = ln 3
+ * A head whose gate is 0 contributes exactly 0, so gmla_decode skips its
+ * attention (its absorbed query rows are left out of the score products). */
+typedef enum gmla_gate_mode {
+  GMLA_GATE_CHANNEL = 0,
+  GMLA_GATE_HEAD = 1,
+  GMLA_GATE_HEAD_TOPK = 2,
+  GMLA_GATE_HEAD_BINARY = 3,
+  GMLA_GATE_HEAD_TERNARY = 4
+} gmla_gate_mode;
 
 typedef struct gmla_config {
   int32_t d_model;
@@ -91,6 +106,7 @@ typedef struct gmla_config {
   int32_t dtype;          /* gmla_dtype */
   int32_t d_cq;           /* low-rank query width d_cq ("精读笔记 03" §5.1: c^Q = W^DQ h,
                              q = W^UQ c^Q; §5.2: q^R = RoPE(W^QR c^Q)); 0 = full-rank query */
+  int32_t gate_topk;      /* k of GMLA_GATE_HEAD_TOPK (1 <= k <= H); ignored otherwise */
 } gmla_config;
 
 typedef struct gmla_weights {

@@ -48,7 +48,7 @@ import numpy as np
 
 __all__ = [
     "params", "sigmoid", "rope", "latent", "project", "project_latent", "project_query", "head_kv",
-    "attention_explicit", "attention_absorbed", "gate", "output",
+    "attention_explicit", "attention_absorbed", "head_gate_values", "gate", "output",
     "prefill", "decode", "kv_elements_per_token", "kv_bytes_per_token",
 ]
 
@@ -71,7 +71,7 @@ def params(inputs: dict) -> dict:
     f = lambda a: None if a is None else np.asarray(a, dtype=np.float64)
     return {
         "H": w.n_heads, "d_h": w.d_h, "d_c": w.d_c, "d_R": w.d_rope,
-        "d_model": w.d_model, "gate_mode": w.gate_mode,
+        "d_model": w.d_model, "gate_mode": w.gate_mode, "gate_topk": w.gate_topk,
         "scale": w.softmax_scale, "rope_base": w.rope_base,
         "W_c": f(inputs["W_c"]), "W_kr": f(inputs.get("W_kr")),
         "W_q": f(inputs.get("W_q")), "W_qr": f(inputs.get("W_qr")),
@@ -242,16 +242,52 @@ def attention_absorbed(p: dict, h: int, q: np.ndarray, qR: np.ndarray,
     return (o, a) if return_weights else o
 
 
+HEAD_GATE_MODES = ("head", "head_topk", "head_binary", "head_ternary")
+
+
+def head_gate_values(p: dict, glogit: np.ndarray) -> np.ndarray:
+    """Per-head gate values [T, H] from the gate logits [T, H].
+
+    * "head": sigmoid(z) ([Gated-MLA concept] "Mathematical Formulation").
+    * "head_topk" ([Gated-MLA concept] "Variants / Extensions", Hard Gating:
+      top-k heads per token): 1 for the k = p["gate_topk"] heads with the
+      largest logits of the token, 0 for the others. Reading: the discrete
+      forward values (the straight-through estimator the page names concerns
+      training only); equal logits go to the lower head index.
+    * "head_binary" (same list, Quantized Gates): 1 where sigmoid(z) >= 1/2,
+      i.e. z >= 0, else 0.
+    * "head_ternary" (same list): sigmoid(z) rounded to the nearest of
+      {0, 1/2, 1} (reading: the three levels of a [0, 1] gate), halfway
+      values rounded up; the cuts are sigmoid(z) = 1/4 and 3/4, z = -+ln 3.
+    """
+    z = np.asarray(glogit, dtype=np.float64)
+    mode = p["gate_mode"]
+    if mode == "head":
+        return sigmoid(z)
+    if mode == "head_topk":
+        k = int(p["gate_topk"])
+        order = np.argsort(-z, axis=1, kind="stable")          # ties: lower index first
+        g = np.zeros_like(z)
+        np.put_along_axis(g, order[:, :k], 1.0, axis=1)
+        return g
+    if mode == "head_binary":
+        return (z >= 0.0).astype(np.float64)
+    if mode == "head_ternary":
+        return np.floor(2.0 * sigmoid(z) + 0.5) / 2.0
+    raise ValueError(mode)
+
+
 def gate(p: dict, glogit: np.ndarray, o_tilde: np.ndarray) -> np.ndarray:
-    """Sigmoid output gate applied to the concatenated heads.
+    """Output gate applied to the concatenated heads.
 
     Per channel ([MLA-gate] §二 boxed equation): Sigmoid(W_g x_t) ⊙ õ_t with
-    G = H*d_h. Per head ([Gated-MLA concept] "Mathematical Formulation"):
-    gates [.., H] broadcast over each head's d_h channels.
+    G = H*d_h. Per head ([Gated-MLA concept] "Mathematical Formulation" and
+    "Variants / Extensions"): gate values [.., H] (head_gate_values) broadcast
+    over each head's d_h channels.
     """
-    g = sigmoid(glogit)
     if p["gate_mode"] == "channel":
-        return g * o_tilde
+        return sigmoid(glogit) * o_tilde
+    g = head_gate_values(p, glogit)
     T = o_tilde.shape[0]
     return (g[:, :, None] * o_tilde.reshape(T, p["H"], p["d_h"])).reshape(T, -1)
 

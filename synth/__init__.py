@@ -25,6 +25,9 @@ Workloads (sizes as named in the problem statement of Gated MLA):
 * ``decode_long_rope_qc``, ``prefill_b4_s4096_qc``: the long-context decode
                          and the batch-4 prefill with a low-rank query,
                          d_cq 1536.
+* ``decode_paged_head_top8``, ``decode_long_rope_top32``: the paged decode and
+                         the long-context decode with hard top-k per-head
+                         gates (8 of 32, 32 of 128 heads).
 
 Drawing order is fixed: x, W_c, W_kr, W_q (or W_dq, W_uq with a compressed
 query), W_qr, W_k, W_v, W_g, b_g, W_o, lengths, page permutation, cache rows.
@@ -54,7 +57,8 @@ class Workload:
     d_c: int
     d_rope: int = 0         # 0 = NoPE
     rope_base: float = 10000.0
-    gate_mode: str = "channel"   # "channel" or "head"
+    gate_mode: str = "channel"   # "channel", or per head: "head", "head_topk", "head_binary", "head_ternary"
+    gate_topk: int = 0           # k of "head_topk"
     gate_bias: bool = False
     gate_bias_var: float = 2.0
     seq_len: int = 0        # prefill: tokens per sequence
@@ -102,6 +106,11 @@ WORKLOADS = {
         name="decode_long_rope", mode="decode", dtype="bf16", batch=8, d_model=7168,
         n_heads=128, d_h=128, d_c=512, d_rope=64, rope_base=10000.0,
         len_law="fixed", len_lo=131072, len_hi=131072),
+    # the long-context decode with 2 sequences instead of 8 (0.3 GB of cache), for ncu captures
+    "decode_long_rope_b2": Workload(
+        name="decode_long_rope_b2", mode="decode", dtype="bf16", batch=2, d_model=7168,
+        n_heads=128, d_h=128, d_c=512, d_rope=64, rope_base=10000.0,
+        len_law="fixed", len_lo=131072, len_hi=131072),
     "decode_paged_head": Workload(
         name="decode_paged_head", mode="decode", dtype="bf16", batch=64, d_model=4096,
         n_heads=32, d_h=128, d_c=512, gate_mode="head", gate_bias=True,
@@ -112,6 +121,17 @@ WORKLOADS = {
         name="decode_long_rope_qc", mode="decode", dtype="bf16", batch=8, d_model=7168,
         n_heads=128, d_h=128, d_c=512, d_rope=64, rope_base=10000.0,
         len_law="fixed", len_lo=131072, len_hi=131072, d_cq=1536),
+    # hard top-k per-head gates (heads outside the top k are skipped in decode):
+    # the paged per-head-gate decode keeping 8 of 32 heads, and the long-context
+    # decode with per-head gates keeping 32 of 128 heads
+    "decode_paged_head_top8": Workload(
+        name="decode_paged_head_top8", mode="decode", dtype="bf16", batch=64, d_model=4096,
+        n_heads=32, d_h=128, d_c=512, gate_mode="head_topk", gate_topk=8, gate_bias=True,
+        len_law="loguniform", len_lo=256, len_hi=32768, paged=True, page_size=64),
+    "decode_long_rope_top32": Workload(
+        name="decode_long_rope_top32", mode="decode", dtype="bf16", batch=8, d_model=7168,
+        n_heads=128, d_h=128, d_c=512, d_rope=64, rope_base=10000.0, gate_mode="head_topk", gate_topk=32,
+        gate_bias=True, len_law="fixed", len_lo=131072, len_hi=131072),
     "prefill_b4_s4096_qc": Workload(
         name="prefill_b4_s4096_qc", mode="prefill", dtype="bf16", batch=4, seq_len=4096,
         d_model=7168, n_heads=64, d_h=128, d_c=512, gate_bias=True, d_cq=1536),

@@ -46,7 +46,7 @@ def make_model(inp, device="cuda"):
     weights["b_g"] = dev(inp["b_g"], torch.float32)
     return GatedMLA(d_model=w.d_model, n_heads=w.n_heads, d_h=w.d_h, d_c=w.d_c, d_rope=w.d_rope,
                     gate_mode=w.gate_mode, softmax_scale=w.softmax_scale, rope_base=w.rope_base,
-                    dtype=dt, weights=weights, d_cq=w.d_cq)
+                    dtype=dt, weights=weights, d_cq=w.d_cq, gate_topk=w.gate_topk)
 
 
 def make_decode_cache(inp, device="cuda", paged=None, capacity=None, fill=float("nan")):

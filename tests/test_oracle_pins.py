@@ -105,6 +105,13 @@ def brute_prefill(inp):
             if bg is not None:
                 logit = [logit[i] + bg[i] for i in range(len(logit))]
             gsig = [1.0 / (1.0 + math.exp(-l)) for l in logit]
+            if w.gate_mode == "head_topk":       # the k largest logits, ties to the lower head
+                ranked = sorted(range(H), key=lambda hh: (-logit[hh], hh))
+                gsig = [1.0 if hh in ranked[:w.gate_topk] else 0.0 for hh in range(H)]
+            elif w.gate_mode == "head_binary":
+                gsig = [1.0 if l >= 0.0 else 0.0 for l in logit]
+            elif w.gate_mode == "head_ternary":  # nearest of 0, 1/2, 1
+                gsig = [min((0.0, 0.5, 1.0), key=lambda v: (abs(v - g_), -v)) for g_ in gsig]
             if w.gate_mode == "channel":
                 gated = [gsig[i] * o_cat[i] for i in range(H * dh)]
             else:
@@ -148,6 +155,82 @@ def test_compressed_query_equals_full_rank_with_the_product_weight(d_rope):
     for k in ("q", "qR", "o", "y"):
         np.testing.assert_allclose(a[k], b[k], rtol=1e-12, atol=1e-13, err_msg=k)
     np.testing.assert_allclose(a["cq"], np.asarray(inp["x"], float) @ p["W_dq"].T, rtol=1e-15)
+
+
+@pytest.mark.parametrize("gate_mode,k", [("head_topk", 1), ("head_topk", 2), ("head_binary", 0),
+                                         ("head_ternary", 0)])
+def test_bruteforce_prefill_hard_and_quantized_head_gates(gate_mode, k):
+    inp = tiny(d_rope=2, gate_mode=gate_mode, gate_topk=k, lengths=(4, 6))
+    p = oracle.params(inp)
+    got = oracle.prefill(p, inp["x"], inp["lengths"])["y"]
+    np.testing.assert_allclose(got, brute_prefill(inp), rtol=1e-12, atol=1e-12)
+
+
+def _hard(gate_mode, k=0, H=6, seed=3, T=40):
+    w = synth.Workload(name="hard", mode="prefill", dtype="f32", batch=1, d_model=8, n_heads=H, d_h=3, d_c=4,
+                       gate_mode=gate_mode, gate_topk=k, gate_bias=True)
+    inp = synth.generate(w, seed=seed, lengths=np.array([T]))
+    p = oracle.params(inp)
+    return inp, p, oracle.project(p, inp["x"], np.arange(T))["glogit"]
+
+
+def test_topk_gates_select_the_k_largest_logits():
+    for k in range(1, 7):
+        inp, p, z = _hard("head_topk", k)
+        g = oracle.head_gate_values(p, z)
+        assert np.all(g.sum(axis=1) == k)
+        for t in range(z.shape[0]):
+            chosen = set(np.flatnonzero(g[t]))
+            assert z[t, list(chosen)].min() >= np.max(np.delete(z[t], list(chosen)), initial=-np.inf)
+    # equal logits: the lower head index wins
+    p = {"gate_mode": "head_topk", "gate_topk": 2}
+    assert np.array_equal(oracle.head_gate_values(p, np.array([[1.0, 3.0, 3.0, 3.0]])), [[0, 1, 1, 0]])
+
+
+def test_topk_with_every_head_is_ungated_mla():
+    inp, p, _ = _hard("head_topk", 6)
+    y = oracle.prefill(p, inp["x"], inp["lengths"])
+    np.testing.assert_allclose(y["y"], oracle.output(p, y["o_tilde"]), rtol=1e-13, atol=1e-15)
+
+
+def test_binary_gate_is_the_saturated_sigmoid():
+    inp, p, z = _hard("head_binary")
+    g = oracle.head_gate_values(p, z)
+    far = np.abs(z) > 1e-2
+    np.testing.assert_array_equal(g[far], oracle.sigmoid(1e5 * z[far]))
+    assert set(np.unique(g)) <= {0.0, 1.0}
+
+
+def test_ternary_gate_is_the_nearest_of_three_levels():
+    inp, p, z = _hard("head_ternary", T=200)
+    g = oracle.head_gate_values(p, z)
+    s = oracle.sigmoid(z)
+    assert set(np.unique(g)) <= {0.0, 0.5, 1.0}
+    assert np.all(np.abs(g - s) <= 0.25 + 1e-15)
+    order = np.argsort(z.ravel())
+    assert np.all(np.diff(g.ravel()[order]) >= 0)               # monotone in the logit
+    cut = math.log(3.0)                                            # sigmoid(+-ln 3) = 3/4, 1/4
+    np.testing.assert_array_equal(oracle.head_gate_values(p, np.array([[-cut - 1e-9, -cut + 1e-9, 0.0,
+                                                                        cut - 1e-9, cut + 1e-9]])),
+                                  [[0.0, 0.5, 0.5, 0.5, 1.0]])
+
+
+@pytest.mark.parametrize("gate_mode,k", [("head_topk", 2), ("head_binary", 0), ("head_ternary", 0)])
+def test_zero_gated_heads_do_not_reach_y(gate_mode, k):
+    """Head skipping is exact: a head whose gate is 0 for a token contributes
+    nothing to that token's y, whatever its attention computes."""
+    inp, p, z = _hard(gate_mode, k)
+    g = oracle.head_gate_values(p, z)
+    y = oracle.prefill(p, inp["x"], inp["lengths"])["y"]
+    for h in range(p["H"]):
+        p2 = dict(p, W_v=p["W_v"].copy(), W_k=p["W_k"].copy())
+        p2["W_v"][h] *= 1e3
+        p2["W_k"][h] *= -7.0
+        y2 = oracle.prefill(p2, inp["x"], inp["lengths"])["y"]
+        off = g[:, h] == 0.0
+        np.testing.assert_allclose(y2[off], y[off], rtol=1e-12, atol=1e-14)
+        if (~off).any():
+            assert np.abs(y2[~off] - y[~off]).max() > 1e-3
 
 
 def test_two_token_closed_form():
