@@ -85,6 +85,9 @@ def _load() -> ctypes.CDLL:
         "gmla_latent_project": (st, [cfgp, wp, P, I, P, P, cp, P, P, P, S, P]),
         "gmla_decode": (st, [cfgp, wp, P, P, cp, P, I, P, P, S, P]),
         "gmla_decode_noalloc": (st, [cfgp, wp, P, P, cp, P, I, P, P]),
+        "gmla_decode_partial": (st, [cfgp, wp, P, P, cp, P, P, I, P, P, S, P]),
+        "gmla_decode_merge": (st, [cfgp, wp, P, I, P, I, P, P, S, P]),
+        "gmla_decode_merge_workspace_size": (S, [cfgp, I]),
         "gmla_prefill": (st, [cfgp, wp, P, P, cp, P, I, I, I, P, P, S, P]),
         "gmla_gate_out": (st, [cfgp, wp, P, I, P, P, P, S, P]),
         "gmla_latent_project_workspace_size": (S, [cfgp, I]),
@@ -132,6 +135,20 @@ def gmla_decode(cfg, w, q, gate_logits, cache, seq_lens, B, o, ws, ws_bytes, str
 def gmla_decode_noalloc(cfg, w, q, gate_logits, cache, seq_lens, B, o, stream):
     return lib.gmla_decode_noalloc(ctypes.byref(cfg), ctypes.byref(w), q, gate_logits, ctypes.byref(cache),
                                    seq_lens, B, o, stream)
+
+
+def gmla_decode_partial(cfg, w, q, gate_logits, cache, seq_starts, seq_ends, B, partial, ws, ws_bytes, stream):
+    return lib.gmla_decode_partial(ctypes.byref(cfg), ctypes.byref(w), q, gate_logits, ctypes.byref(cache),
+                                   seq_starts, seq_ends, B, partial, ws, ws_bytes, stream)
+
+
+def gmla_decode_merge(cfg, w, partials, R, gate_logits, B, o, ws, ws_bytes, stream):
+    return lib.gmla_decode_merge(ctypes.byref(cfg), ctypes.byref(w), partials, R, gate_logits, B, o, ws, ws_bytes,
+                                 stream)
+
+
+def gmla_decode_merge_workspace_size(cfg, B):
+    return lib.gmla_decode_merge_workspace_size(ctypes.byref(cfg), B)
 
 
 def gmla_prefill(cfg, w, q, gate_logits, cache, cu_seqlens, B, T, max_seqlen, o, ws, ws_bytes, stream):

@@ -68,6 +68,11 @@ __device__ __forceinline__ int block_excl_scan(int v, int* s_warp, int* total) {
   return r;
 }
 
+// 128-token tiles that cover positions [start, L) of a sequence.
+__device__ __forceinline__ int seq_tiles(int L, int start) {
+  return L > start ? (L + kTileTok - 1) / kTileTok - start / kTileTok : 0;
+}
+
 // Tiles of 128 tokens of all sequences, concatenated, are cut into G equal
 // ranges (one per CTA of a head group). A segment is the part of one sequence
 // inside one range; seg_info = {sequence, first tile, end tile, CTA}.
@@ -81,11 +86,12 @@ __device__ void decode_plan_block(const DecodeArgs& a) {
   __syncthreads();
   for (int b = tid; b < a.B; b += blockDim.x) {
     int L = a.seq_lens[b];
-    if (L < 0 || L > limit || b >= a.cache.batch) {
+    const int s0 = a.seq_starts ? a.seq_starts[b] : 0;
+    if (L < 0 || L > limit || b >= a.cache.batch || s0 < 0) {
       report_status(a.status, kStatusRange);
       L = 0;
     }
-    atomicAdd(&s_sum, (L + kTileTok - 1) / kTileTok);
+    atomicAdd(&s_sum, seq_tiles(L, s0));
   }
   __syncthreads();
   const int total = s_sum;
@@ -94,8 +100,10 @@ __device__ void decode_plan_block(const DecodeArgs& a) {
   for (int base = 0; base < a.B; base += blockDim.x) {
     const int b = base + tid;
     int L = b < a.B ? a.seq_lens[b] : 0;
-    if (L < 0 || L > limit || b >= a.cache.batch) L = 0;
-    const int t = (L + kTileTok - 1) / kTileTok;
+    const int s0 = (b < a.B && a.seq_starts) ? a.seq_starts[b] : 0;
+    if (L < 0 || L > limit || b >= a.cache.batch || s0 < 0) L = 0;
+    const int t = seq_tiles(L, s0);
+    const int ts = s0 / kTileTok;   // first tile of the sequence's range
     int tsum, ssum;
     const int P = tile_carry + block_excl_scan(t, s_warp, &s_total);
     tsum = s_total;
@@ -111,7 +119,7 @@ __device__ void decode_plan_block(const DecodeArgs& a) {
       for (int k = 0; k < nseg; ++k) {
         const int g = g_first + k;
         const int lo = max(P, g * tpc), hi = min(P + t, (g + 1) * tpc);
-        a.seg_info[S + k] = make_int4(b, lo - P, hi - P, g);
+        a.seg_info[S + k] = make_int4(b, ts + lo - P, ts + hi - P, g);
         if (g * tpc >= P) a.cta_first_seg[g] = S + k;   // range g starts inside sequence b
       }
     }
@@ -543,6 +551,7 @@ __global__ void __launch_bounds__(64 + 128 * (HG >= 32 ? 2 : 1), 1) decode_attn_
     for (int si = seg_lo; si < seg_hi; ++si) {
       const int4 sg = a.seg_info[si];
       const int L = a.seq_lens[sg.x];
+      const int S0 = a.seq_starts ? a.seq_starts[sg.x] : 0;
       const int hv = seg_heads(a, sg.x, hg, heads_valid);
       if (hv == 0) continue;
       float m[HT], lsum[HT];
@@ -559,7 +568,9 @@ __global__ void __launch_bounds__(64 + 128 * (HG >= 32 ? 2 : 1), 1) decode_attn_
         // again for P, so no thread holds all its heads' scores at once.
         const uint32_t tS = tmem + (ntile & 1) * HG + lane_off + h0;
         const int valid = min(kTileTok, L - t * kTileTok);
-        const bool rv = row < valid;
+        // rows of the tile outside [start, L): past the end, or (a context-parallel
+        // shard) before the first position this call attends to
+        const bool rv = row < valid && t * kTileTok + row >= S0;
         auto load16 = [&](int c, float (&x)[16]) {
           uint32_t v[16];
           tmem_ld16(tS + c, v);
@@ -744,6 +755,12 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(DecodeArgs a) {
     // slot -> head; a head whose gate is 0 was skipped: its latent output is 0
     h = a.head_of_slot[static_cast<int64_t>(b) * a.H + slot];
     if (slot >= a.n_act[b]) {
+      if (a.partial_out) {   // an empty partial: O = 0, log-sum-exp -inf
+        float* dst = a.partial_out + (static_cast<int64_t>(b) * a.H + h) * (kDc + kPartialPad);
+        for (int j = threadIdx.x; j < kDc + kPartialPad; j += blockDim.x)
+          dst[j] = j == kDc ? -__int_as_float(0x7f800000) : 0.f;
+        return;
+      }
       __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.olat) + (static_cast<int64_t>(h) * a.B + b) * kDc;
       for (int j = threadIdx.x; j < kDc; j += blockDim.x) dst[j] = __float2bfloat16_rn(0.f);
       return;
@@ -773,9 +790,66 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(DecodeArgs a) {
     mx = mn;
   }
   const float inv = (s1 > s0 && l > 0.f) ? 1.f / l : 0.f;
+  if (a.partial_out) {
+    // context-parallel share: normalised O_lat of this share and its log-sum-exp
+    // (log2 domain), merged across shares by decode_merge_ranks
+    float* dst = a.partial_out + (static_cast<int64_t>(b) * a.H + h) * (kDc + kPartialPad);
+#pragma unroll
+    for (int j = 0; j < kDc / 128; ++j) dst[j * 128 + threadIdx.x] = acc[j] * inv;
+    if (threadIdx.x < kPartialPad)
+      dst[kDc + threadIdx.x] = threadIdx.x == 0 ? ((l > 0.f) ? mx + __log2f(l) : -__int_as_float(0x7f800000)) : 0.f;
+    return;
+  }
   __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.olat) + (static_cast<int64_t>(h) * a.B + b) * kDc;
 #pragma unroll
   for (int j = 0; j < kDc / 128; ++j) dst[j * 128 + threadIdx.x] = __float2bfloat16_rn(acc[j] * inv);
+}
+
+// ---------------------------------------------------------------------------
+// 5. context-parallel merge: the shares of one sequence's cache held by R
+//    ranks each give (O_r normalised, lse_r); O = sum_r 2^(lse_r - M) O_r /
+//    sum_r 2^(lse_r - M), M = max_r lse_r. One block per (head, sequence).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(128) decode_merge_ranks_kernel(MergeRanksArgs a) {
+  if (threadIdx.x == 0) griddep_launch_dependents();
+  griddep_wait();
+  const int h = blockIdx.x, b = blockIdx.y;
+  const float NEG_INF = -__int_as_float(0x7f800000);
+  const int64_t row = static_cast<int64_t>(b) * a.H + h;
+  const int64_t rank_stride = static_cast<int64_t>(a.B) * a.H * (kDc + kPartialPad);
+  float mx = NEG_INF, wsum = 0.f;
+  float acc[kDc / 128];
+#pragma unroll
+  for (int j = 0; j < kDc / 128; ++j) acc[j] = 0.f;
+  for (int r = 0; r < a.R; ++r) {
+    const float* src = a.partials + r * rank_stride + row * (kDc + kPartialPad);
+    const float lse = __ldcg(src + kDc);
+    if (lse == NEG_INF) continue;   // an empty share
+    float o[kDc / 128];
+#pragma unroll
+    for (int j = 0; j < kDc / 128; ++j) o[j] = __ldcg(src + j * 128 + threadIdx.x);
+    const float mn = fmaxf(mx, lse);
+    const float a_old = (mx == NEG_INF) ? 0.f : ex2_approx(mx - mn);
+    const float a_new = ex2_approx(lse - mn);
+    wsum = wsum * a_old + a_new;
+#pragma unroll
+    for (int j = 0; j < kDc / 128; ++j) acc[j] = acc[j] * a_old + o[j] * a_new;
+    mx = mn;
+  }
+  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+  __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.olat) + (static_cast<int64_t>(h) * a.B + b) * kDc;
+#pragma unroll
+  for (int j = 0; j < kDc / 128; ++j) dst[j * 128 + threadIdx.x] = __float2bfloat16_rn(acc[j] * inv);
+  if (a.gate_hard && threadIdx.x == 0)
+    a.gvals[row] = head_gate(a.gate_logits + static_cast<int64_t>(b) * a.H, a.H, h, a.gate_mode, a.gate_topk);
+}
+
+cudaError_t launch_decode_merge_ranks(const MergeRanksArgs& a, cudaStream_t st) {
+  if (a.B == 0) return cudaSuccess;
+  prof_begin(st, "decode_merge_ranks");
+  cudaError_t e = launch_pdl(decode_merge_ranks_kernel, dim3(a.H, a.B), dim3(128), 0, st, 1, a);
+  prof_end(st);
+  return e;
 }
 
 // ---------------------------------------------------------------------------

@@ -496,9 +496,12 @@ gmla_status gmla_latent_project(const gmla_config* cfg, const gmla_weights* w, c
 }
 
 // ---------------------------------------------------------------------------
-gmla_status gmla_decode(const gmla_config* cfg, const gmla_weights* w, const void* q, const float* gate_logits,
-                        const gmla_cache* cache, const int32_t* seq_lens, int32_t B, void* o_gated,
-                        void* workspace, size_t workspace_bytes, void* stream) {
+// gmla_decode, and the context-parallel share of it (positions [seq_starts[b],
+// seq_lens[b]) written as partials instead of o_gated) for gmla_decode_partial.
+static gmla_status decode_impl(const gmla_config* cfg, const gmla_weights* w, const void* q,
+                               const float* gate_logits, const gmla_cache* cache, const int32_t* seq_starts,
+                               const int32_t* seq_lens, int32_t B, void* o_gated, float* partial_out,
+                               void* workspace, size_t workspace_bytes, void* stream) {
   GMLA_TRY(check_cfg(cfg));
   if (!w) return fail(GMLA_ERR_INVALID_ARG, "weights is NULL");
   if (B < 0) return fail(GMLA_ERR_INVALID_ARG, "B < 0");
@@ -511,14 +514,21 @@ gmla_status gmla_decode(const gmla_config* cfg, const gmla_weights* w, const voi
   if (B > cache->batch) return fail(GMLA_ERR_INVALID_ARG, "B (%d) exceeds cache.batch (%d)", B, cache->batch);
   GMLA_TRY(check_ptr(q, "q"));
   GMLA_TRY(check_ptr(seq_lens, "seq_lens"));
-  GMLA_TRY(check_ptr(o_gated, "o_gated"));
+  GMLA_TRY(check_ptr(seq_starts, "seq_starts", false));
+  if (partial_out) {
+    GMLA_TRY(check_ptr(partial_out, "partial"));
+  } else {
+    GMLA_TRY(check_ptr(o_gated, "o_gated"));
+  }
   GMLA_TRY(check_ptr(gate_logits, "gate_logits", false));
   GMLA_TRY(check_ptr(w->W_k, "W_k"));
-  GMLA_TRY(check_ptr(w->W_v, "W_v"));
+  if (!partial_out) GMLA_TRY(check_ptr(w->W_v, "W_v"));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const CacheView cv = cache_view(cfg, cache);
   int* status = static_cast<int*>(workspace);
 
+  if (cfg->dtype == GMLA_FP32 && (partial_out || seq_starts))
+    return fail(GMLA_ERR_UNSUPPORTED, "context-parallel decode covers the bf16 path");
   if (cfg->dtype == GMLA_FP32) {
     AttnF32Args a{};
     a.q = static_cast<const float*>(q);
@@ -597,6 +607,8 @@ gmla_status gmla_decode(const gmla_config* cfg, const gmla_weights* w, const voi
   a.gvals = reinterpret_cast<float*>(ws + L.off_gvals);
   a.head_of_slot = reinterpret_cast<int32_t*>(ws + L.off_hslot);
   a.n_act = reinterpret_cast<int32_t*>(ws + L.off_nact);
+  a.seq_starts = seq_starts;
+  a.partial_out = partial_out;
   a.olat = ws + L.off_olat;
   const SwapPlan& sp = L.gemm_plan;
   a.gemm_counters = nullptr;
@@ -630,8 +642,94 @@ gmla_status gmla_decode(const gmla_config* cfg, const gmla_weights* w, const voi
   g.status = status;
 
   cudaError_t e = launch_decode_bf16(a, st);
-  if (e == cudaSuccess) e = launch_gemm_bf16(g, true, sp.bn, sp.ttiles, st, "gemm_wv_gate");
+  if (e == cudaSuccess && !partial_out) e = launch_gemm_bf16(g, true, sp.bn, sp.ttiles, st, "gemm_wv_gate");
   return e == cudaSuccess ? GMLA_OK : cuda_fail(e, "decode");
+}
+
+gmla_status gmla_decode(const gmla_config* cfg, const gmla_weights* w, const void* q, const float* gate_logits,
+                        const gmla_cache* cache, const int32_t* seq_lens, int32_t B, void* o_gated,
+                        void* workspace, size_t workspace_bytes, void* stream) {
+  return decode_impl(cfg, w, q, gate_logits, cache, nullptr, seq_lens, B, o_gated, nullptr, workspace,
+                     workspace_bytes, stream);
+}
+
+gmla_status gmla_decode_partial(const gmla_config* cfg, const gmla_weights* w, const void* q,
+                                const float* gate_logits, const gmla_cache* cache, const int32_t* seq_starts,
+                                const int32_t* seq_ends, int32_t B, float* partial, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+  if (!partial && B > 0) return fail(GMLA_ERR_INVALID_ARG, "partial is NULL");
+  return decode_impl(cfg, w, q, gate_logits, cache, seq_starts, seq_ends, B, nullptr, partial, workspace,
+                     workspace_bytes, stream);
+}
+
+size_t gmla_decode_merge_workspace_size(const gmla_config* cfg, int32_t B) {
+  if (!cfg_valid(cfg) || B < 0) return 256;
+  const size_t olat = align256(static_cast<size_t>(cfg->n_heads) * B * cfg->d_c * 2);
+  const size_t gv = align256(static_cast<size_t>(B) * cfg->n_heads * 4);
+  return 256 + olat + gv;
+}
+
+gmla_status gmla_decode_merge(const gmla_config* cfg, const gmla_weights* w, const float* partials, int32_t R,
+                              const float* gate_logits, int32_t B, void* o_gated, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  GMLA_TRY(check_cfg(cfg));
+  if (!w) return fail(GMLA_ERR_INVALID_ARG, "weights is NULL");
+  if (B < 0 || R < 1) return fail(GMLA_ERR_INVALID_ARG, "B < 0 or R < 1");
+  const size_t need = gmla_decode_merge_workspace_size(cfg, B);
+  if (!workspace || workspace_bytes < need)
+    return fail(GMLA_ERR_WORKSPACE, "decode_merge needs %zu workspace bytes, got %zu", need, workspace_bytes);
+  GMLA_TRY(check_ptr(workspace, "workspace"));
+  if (B == 0) return GMLA_OK;
+  if (cfg->dtype != GMLA_BF16 || cfg->d_c != 512 || cfg->d_h % 128)
+    return fail(GMLA_ERR_UNSUPPORTED, "context-parallel merge covers bf16 with d_c = 512 and d_h %% 128 == 0");
+  GMLA_TRY(check_ptr(partials, "partials"));
+  GMLA_TRY(check_ptr(o_gated, "o_gated"));
+  GMLA_TRY(check_ptr(gate_logits, "gate_logits", false));
+  GMLA_TRY(check_ptr(w->W_v, "W_v"));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const int H = cfg->n_heads, HD = H * cfg->d_h, G = gate_width(cfg);
+  void* olat = ws + 256;
+  float* gvals = reinterpret_cast<float*>(ws + 256 + align256(static_cast<size_t>(H) * B * cfg->d_c * 2));
+  MergeRanksArgs m{};
+  m.partials = partials;
+  m.R = R;
+  m.B = B;
+  m.H = H;
+  m.olat = olat;
+  m.gate_logits = gate_logits;
+  m.gate_mode = cfg->gate_mode;
+  m.gate_topk = cfg->gate_topk;
+  m.gate_hard = (gate_is_hard(cfg->gate_mode) && gate_logits) ? 1 : 0;
+  m.gvals = gvals;
+  cudaError_t e = launch_decode_merge_ranks(m, st);
+  if (e != cudaSuccess) return cuda_fail(e, "decode_merge");
+  // o = gate ⊙ W_v^(h) O_lat^(h), the same tensor-core GEMM as gmla_decode's
+  const SwapPlan sp = gemm_swap_plan(HD / 128, B, cfg->d_c, num_sms());
+  GemmArgs g{};
+  if (!make_tmap_2d(&g.act, olat, cfg->d_c, static_cast<uint64_t>(H) * B, static_cast<uint64_t>(cfg->d_c) * 2, 64,
+                    sp.bn, true) ||
+      !make_tmap_2d(&g.wt[0], w->W_v, cfg->d_c, HD, static_cast<uint64_t>(cfg->d_c) * 2, 64, 128, true))
+    return fail(GMLA_ERR_CUDA, "tensor maps for the W_v product failed");
+  g.epi[0] = plain_seg(o_gated, HD, 1 << 30, 0, 0, false, nullptr, false, false);
+  g.epi[0].gate = m.gate_hard ? gvals : gate_logits;
+  g.epi[0].gate_value = m.gate_hard;
+  g.epi[0].gate_stride = G;
+  g.epi[0].gate_div = cfg->gate_mode == GMLA_GATE_CHANNEL ? 1 : cfg->d_h;
+  g.seg_rows[0] = HD;
+  g.seg_tile_begin[0] = 0;
+  g.seg_tile_begin[1] = HD / 128;
+  g.n_seg = 1;
+  g.T = B;
+  g.K = cfg->d_c;
+  g.row_mode = 2;
+  g.rows_per_group = cfg->d_h;
+  g.act_group_stride = B;
+  g.splits = sp.splits;
+  g.kb_per_split = sp.kb_per_split;
+  g.status = static_cast<int*>(workspace);
+  e = launch_gemm_bf16(g, true, sp.bn, sp.ttiles, st, "gemm_wv_gate");
+  return e == cudaSuccess ? GMLA_OK : cuda_fail(e, "decode_merge: W_v");
 }
 
 // ---------------------------------------------------------------------------
@@ -687,7 +785,8 @@ gmla_status gmla_prefill(const gmla_config* cfg, const gmla_weights* w, const vo
     return e == cudaSuccess ? GMLA_OK : cuda_fail(e, "prefill (fp32)");
   }
 
-  if (cfg->d_rope != 0) return fail(GMLA_ERR_UNSUPPORTED, "bf16 prefill covers NoPE (d_rope = 0)");
+  if (cfg->d_rope != 0 && cfg->d_rope != 64)
+    return fail(GMLA_ERR_UNSUPPORTED, "bf16 prefill covers NoPE or decoupled RoPE of 64 dims");
   if (cfg->d_h != 128) return fail(GMLA_ERR_UNSUPPORTED, "bf16 prefill covers d_h = 128");
   if (cfg->d_c % 64) return fail(GMLA_ERR_UNSUPPORTED, "bf16 prefill needs d_c %% 64 == 0");
   const int H = cfg->n_heads, HD = H * cfg->d_h;
@@ -730,6 +829,14 @@ gmla_status gmla_prefill(const gmla_config* cfg, const gmla_weights* w, const vo
       !make_tmap_2d(&p.k_map, Kbuf, HD, T, static_cast<uint64_t>(HD) * 2, 64, 128, true) ||
       !make_tmap_2d(&p.v_map, Vbuf, HD, T, static_cast<uint64_t>(HD) * 2, 64, 128, true))
     return fail(GMLA_ERR_CUDA, "tensor maps for prefill attention failed");
+  // decoupled RoPE: k^R is read from the cache rows (its last d_R columns)
+  if (cfg->d_rope &&
+      !make_tmap_2d(&p.kr_map, cache->data, cv.row, static_cast<uint64_t>(cache->batch) * cache->capacity,
+                    static_cast<uint64_t>(cv.row) * 2, 64, 128, true))
+    return fail(GMLA_ERR_CUDA, "tensor map for the cached k^R failed");
+  p.d_c = cfg->d_c;
+  p.d_rope = cfg->d_rope;
+  p.cache_capacity = cache->capacity;
   p.gate_logits = gate_logits;
   p.o = o_gated;
   p.cu_seqlens = cu_seqlens;

@@ -90,7 +90,24 @@ struct DecodeArgs {
   float* gvals;              // workspace: [B, H] gate values
   int32_t* head_of_slot;     // workspace: [B, H]
   int32_t* n_act;            // workspace: [B] heads whose gate is not 0
+  // context-parallel share: attend to positions [seq_starts[b], seq_lens[b]) only
+  // (null: from 0), and write per-(sequence, head) partials instead of O_lat
+  const int32_t* seq_starts;
+  float* partial_out;        // [B, H, d_c + 4]: O_lat / l, then log2-domain m + log2 l
 };
+
+// Cross-rank merge of context-parallel partials into O_lat (bf16 [H, B, d_c]),
+// plus the gate values of hard / quantised per-head gates.
+struct MergeRanksArgs {
+  const float* partials;     // [R, B, H, d_c + 4]
+  int32_t R, B, H;
+  void* olat;                // [H, B, d_c] bf16
+  const float* gate_logits;  // [B, H] (hard gates only) or null
+  int32_t gate_mode, gate_topk, gate_hard;
+  float* gvals;              // [B, H]
+};
+cudaError_t launch_decode_merge_ranks(const MergeRanksArgs& a, cudaStream_t st);
+constexpr int kPartialPad = 4;   // floats after the d_c values of a partial row
 
 struct DecodeLayout {
   size_t off_qa, off_opart, off_ml, off_seg, off_seqfirst, off_ctafirst, off_olat, off_gemm;
@@ -142,6 +159,8 @@ struct PrefillArgs {
   CUtensorMap q_map;         // 2D [T, H*(d_h+d_R)] bf16
   CUtensorMap k_map;         // 2D [T, H*d_h] bf16
   CUtensorMap v_map;         // 2D [T, H*d_h] bf16
+  CUtensorMap kr_map;        // 2D cache rows [batch*capacity, d_c + d_R] bf16 (decoupled RoPE only)
+  int32_t d_c, d_rope, cache_capacity;
   const float* gate_logits;  // [T, G] or null
   void* o;                   // [T, H*d_h]
   const int32_t* cu_seqlens;

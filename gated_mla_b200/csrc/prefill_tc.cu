@@ -27,11 +27,24 @@ namespace {
 constexpr int kBQ = 128;          // queries per tile
 constexpr int kBK = 128;          // keys per tile
 constexpr int kD = 128;           // head dim
+constexpr int kDR = 64;           // decoupled RoPE dims (one box) when present
 constexpr int kBox = 128 * 128;   // one [128 rows x 64] bf16 box: 16 KB
 constexpr int kTile = 2 * kBox;   // [128 rows x 128] bf16
 constexpr int kStages = 2;
-constexpr int kSmem = 2 * kTile + kStages * 2 * kTile + 1024 + 256;
 constexpr uint32_t kTmemCols = 512;   // per tile: S/P 128 columns + O 128 columns
+
+// NoPE: two query tiles per CTA, Q and K rows of d_h = 128 (2 boxes).
+// Decoupled RoPE: each Q and K row grows by the 64 rotated dims (a third box:
+// q^R of the head; k^R shared by all heads, read from the cache rows), and one
+// query tile per CTA keeps the stages in shared memory.
+template <bool kRope>
+struct PfCfg {
+  static constexpr int kQKBoxes = kRope ? 3 : 2;
+  static constexpr int kQTile = kQKBoxes * kBox;
+  static constexpr int kKTile = kQKBoxes * kBox;
+  static constexpr int kQTiles = kRope ? 1 : 2;
+  static constexpr int kSmem = kQTiles * kQTile + kStages * (kKTile + kTile) + 1024 + 256;
+};
 
 struct PfBars {
   uint64_t q_full;
@@ -43,12 +56,14 @@ struct PfBars {
 };
 }  // namespace
 
+template <bool kRope>
 __global__ void __launch_bounds__(320, 1) prefill_attn_kernel(const __grid_constant__ PrefillArgs a) {
+  using C = PfCfg<kRope>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;                             // [tile A, tile B]
-  uint8_t* sK = sQ + 2 * kTile;                   // [stage]
-  uint8_t* sV = sK + kStages * kTile;             // [stage]
+  uint8_t* sK = sQ + C::kQTiles * C::kQTile;      // [stage]
+  uint8_t* sV = sK + kStages * C::kKTile;         // [stage]
   PfBars* bars = reinterpret_cast<PfBars*>(sV + kStages * kTile);
   volatile int* abort_flag = &bars->abort;
 
@@ -57,13 +72,14 @@ __global__ void __launch_bounds__(320, 1) prefill_attn_kernel(const __grid_const
   const int beg = a.cu_seqlens[b];
   const int len = a.cu_seqlens[b + 1] - beg;
   const int n_qt = (len + kBQ - 1) / kBQ;
-  const int pair = (n_qt + 1) / 2 - 1 - static_cast<int>(blockIdx.x);   // long rows first
+  // NoPE: a pair of query tiles per CTA; RoPE: one (tile B absent)
+  const int pair = (kRope ? n_qt : (n_qt + 1) / 2) - 1 - static_cast<int>(blockIdx.x);   // long rows first
   if (pair < 0) return;
-  const int qtA = 2 * pair, qtB = 2 * pair + 1;
-  const bool hasB = qtB < n_qt;
+  const int qtA = kRope ? pair : 2 * pair, qtB = qtA + 1;
+  const bool hasB = !kRope && qtB < n_qt;
   const int n_kv = hasB ? qtB + 1 : qtA + 1;     // causal: key tiles 0..last query tile
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int dq = a.d_h;                          // NoPE: q row is d_h wide per head
+  const int dq = a.d_h + (kRope ? kDR : 0);      // q row of a head: [q | q^R]
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
@@ -96,22 +112,26 @@ __global__ void __launch_bounds__(320, 1) prefill_attn_kernel(const __grid_const
       tma_prefetch_desc(&a.k_map);
       tma_prefetch_desc(&a.v_map);
       const uint64_t pol = l2_evict_last();
-      mbar_arrive_expect_tx(&bars->q_full, (hasB ? 2 : 1) * kTile);
+      mbar_arrive_expect_tx(&bars->q_full, (hasB ? 2 : 1) * C::kQTile);
       for (int x = 0; x < (hasB ? 2 : 1); ++x)
-        for (int kb = 0; kb < 2; ++kb)
-          tma_load_2d(&a.q_map, &bars->q_full, sQ + x * kTile + kb * kBox, h * dq + kb * 64,
+        for (int kb = 0; kb < C::kQKBoxes; ++kb)
+          tma_load_2d(&a.q_map, &bars->q_full, sQ + x * C::kQTile + kb * kBox, h * dq + kb * 64,
                       beg + (qtA + x) * kBQ, pol);
       int issued = 0;
       for (int j = 0; j < n_kv; ++j) {
         const int st = j % kStages;
         if (j >= kStages && !mbar_wait(&bars->kv_empty[st], ((j / kStages) & 1) ^ 1, abort_flag, a.status)) break;
-        mbar_arrive_expect_tx(&bars->kv_full[st], 2 * kTile);
+        mbar_arrive_expect_tx(&bars->kv_full[st], C::kKTile + kTile);
         for (int kb = 0; kb < 2; ++kb) {
-          tma_load_2d(&a.k_map, &bars->kv_full[st], sK + st * kTile + kb * kBox, h * kD + kb * 64,
+          tma_load_2d(&a.k_map, &bars->kv_full[st], sK + st * C::kKTile + kb * kBox, h * kD + kb * 64,
                       beg + j * kBK, pol);
           tma_load_2d(&a.v_map, &bars->kv_full[st], sV + st * kTile + kb * kBox, h * kD + kb * 64,
                       beg + j * kBK, pol);
         }
+        // k^R of these keys (rotated, shared by all heads): the RoPE columns of the cache rows
+        if (kRope)
+          tma_load_2d(&a.kr_map, &bars->kv_full[st], sK + st * C::kKTile + 2 * kBox, a.d_c,
+                      b * a.cache_capacity + j * kBK, pol);
         ++issued;
       }
       if (*abort_flag) {
@@ -125,10 +145,10 @@ __global__ void __launch_bounds__(320, 1) prefill_attn_kernel(const __grid_const
       constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);   // Q K-major, K K-major
       constexpr uint32_t idO = idesc_bf16_f32(128, 128, false, true);    // P from TMEM, V MN-major
       const uint32_t qa = smem_u32(sQ), ka = smem_u32(sK), va = smem_u32(sV);
-      auto issue_s = [&](int x, int j) {   // S_x = Q_x K_j^T
-        const uint32_t kbase = ka + (j % kStages) * kTile, qbase = qa + x * kTile;
+      auto issue_s = [&](int x, int j) {   // S_x = Q_x K_j^T (+ Q^R_x K^R_j^T)
+        const uint32_t kbase = ka + (j % kStages) * C::kKTile, qbase = qa + x * C::kQTile;
 #pragma unroll
-        for (int k = 0; k < kD / 16; ++k) {
+        for (int k = 0; k < C::kQKBoxes * 4; ++k) {
           const int kb = k >> 2, kk = k & 3;
           umma_bf16(tmem + 256 * x, sdesc_sw128(qbase + kb * kBox + kk * 32, 16, 1024),
                     sdesc_sw128(kbase + kb * kBox + kk * 32, 16, 1024), idS, k != 0);
@@ -398,15 +418,22 @@ __global__ void __launch_bounds__(320, 1) prefill_attn_kernel(const __grid_const
   }
 }
 
-cudaError_t launch_prefill_attn_bf16(const PrefillArgs& a, cudaStream_t st) {
-  if (a.d_h != kD) return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(prefill_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+template <bool kRope>
+static cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t st) {
+  using C = PfCfg<kRope>;
+  auto k = prefill_attn_kernel<kRope>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
-  const int pairs = (a.q_tiles_per_seq + 1) / 2;
+  const int ctas = kRope ? a.q_tiles_per_seq : (a.q_tiles_per_seq + 1) / 2;
   prof_begin(st, "prefill_attn");
-  e = launch_pdl(prefill_attn_kernel, dim3(pairs, a.H, a.B), dim3(320), kSmem, st, 1, a);
+  e = launch_pdl(k, dim3(ctas, a.H, a.B), dim3(320), C::kSmem, st, 1, a);
   prof_end(st);
   return e;
+}
+
+cudaError_t launch_prefill_attn_bf16(const PrefillArgs& a, cudaStream_t st) {
+  if (a.d_h != kD || (a.d_rope != 0 && a.d_rope != kDR)) return cudaErrorInvalidValue;
+  return a.d_rope ? launch_prefill<true>(a, st) : launch_prefill<false>(a, st);
 }
 
 }  // namespace gmla

@@ -243,6 +243,45 @@ GMLA_API gmla_status gmla_decode_noalloc(const gmla_config* cfg, const gmla_weig
                                          const gmla_cache* cache, const int32_t* seq_lens,
                                          int32_t B, void* o_gated, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * Context-parallel decode: one sequence's cache split across R GPUs (ranks),
+ * each holding a range of its positions. The softmax over all L rows is the
+ * one of "Gated MLA 计算公式" §二; it decomposes over disjoint ranges: a range
+ * r gives O_r = sum_{s in r} e^{z_s - M_r} c_s / l_r and the log-sum-exp
+ * lse_r = M_r + log l_r, and O_lat = sum_r e^{lse_r - M} O_r / sum_r e^{lse_r - M}
+ * with M = max_r lse_r. Each rank calls gmla_decode_partial on its rows, the
+ * partials of all ranks are gathered (one NCCL all-gather of
+ * R x B x H x (d_c + 4) floats, outside the library), and any rank calls
+ * gmla_decode_merge, which applies W_v and the gate as gmla_decode does.
+ *
+ * gmla_decode_partial — gmla_decode restricted to cached positions
+ * [seq_starts[b], seq_ends[b]) of each sequence (bf16 path).
+ *   q, gate_logits, cache, B, workspace: as gmla_decode (the workspace size is
+ *                gmla_decode_workspace_size(cfg, B)); gate logits only matter
+ *                for hard / quantised gates, whose zero-gated heads are skipped
+ *   seq_starts   [B] int32 or NULL (= 0): first position this rank attends to;
+ *                the rows of the cache below it are never used
+ *   seq_ends     [B] int32: one past the last position (<= the cache's rows)
+ *   partial      [B, H, d_c + 4] fp32: per (sequence, head) the normalised
+ *                latent output O_r (d_c values), then lse_r in log2 units
+ *                (-inf for an empty range or a skipped head), then 3 zeros
+ * gmla_decode_merge — merges R partials into o_gated.
+ *   partials     [R, B, H, d_c + 4] fp32 (the gathered partials, rank-major)
+ *   gate_logits  [B, G] fp32 or NULL (ungated), as gmla_decode
+ *   o_gated      [B, H*d_h]
+ *   workspace    gmla_decode_merge_workspace_size(cfg, B) bytes
+ * ------------------------------------------------------------------------- */
+GMLA_API gmla_status gmla_decode_partial(const gmla_config* cfg, const gmla_weights* w,
+                                         const void* q, const float* gate_logits,
+                                         const gmla_cache* cache, const int32_t* seq_starts,
+                                         const int32_t* seq_ends, int32_t B, float* partial,
+                                         void* workspace, size_t workspace_bytes, void* stream);
+GMLA_API gmla_status gmla_decode_merge(const gmla_config* cfg, const gmla_weights* w,
+                                       const float* partials, int32_t R, const float* gate_logits,
+                                       int32_t B, void* o_gated, void* workspace,
+                                       size_t workspace_bytes, void* stream);
+GMLA_API size_t gmla_decode_merge_workspace_size(const gmla_config* cfg, int32_t B);
+
 /* Scratch sizes in bytes (0 is never returned; 256-byte aligned). An invalid
  * configuration or a negative size gets 256 (the calls themselves then fail
  * with GMLA_ERR_INVALID_ARG). */

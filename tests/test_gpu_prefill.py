@@ -25,6 +25,10 @@ def _check(inp, gpu, tol, rows=None):
     starts = np.concatenate([[0], np.cumsum(inp["lengths"])])
     for b, L in enumerate(inp["lengths"]):
         assert_close(cache[b, :L, :w.d_c], ref["c"][starts[b]:starts[b] + L], tol, f"cached latents seq {b}")
+        if w.d_rope:
+            assert_close(cache[b, :L, w.d_c:], ref["kR"][starts[b]:starts[b] + L], tol, f"cached k^R seq {b}")
+    if w.d_rope:
+        assert_close(gpu["q"][idx][:, :, dh:], ref["qR"], tol, "q^R (rotated)")
 
 
 def test_prefill_tiny_fp32_full_config():
@@ -48,6 +52,22 @@ def test_prefill_bf16_ragged_tiles():
 def test_prefill_bf16_long_sequence_many_heads():
     inp = synth.generate(synth.workload("prefill_b4_s4096", batch=2, d_model=1024, n_heads=16), seed=2,
                          lengths=np.array([1000, 700]))
+    _check(inp, run_prefill(inp), BF16_TOL)
+
+
+def test_prefill_bf16_decoupled_rope_ragged():
+    """Decoupled RoPE ("精读笔记 03" §5.2): scores add q^R . k^R with k^R read from
+    the cache rows; lengths 1, 127, 128, 129, 300."""
+    inp = synth.generate(synth.workload("prefill_b4_s4096", batch=5, d_model=512, n_heads=4, d_rope=64), seed=3,
+                         lengths=np.array([1, 127, 128, 129, 300]))
+    _check(inp, run_prefill(inp), BF16_TOL)
+
+
+def test_prefill_bf16_decoupled_rope_long_positions():
+    """A 1500-token prompt of the long-context shape (d_c 512 + RoPE 64, base
+    10000) with 16 heads: angles of positions up to 1499."""
+    inp = synth.generate(synth.workload("prefill_b4_s4096", batch=2, d_model=1024, n_heads=16, d_rope=64,
+                                        gate_bias=False), seed=4, lengths=np.array([1500, 260]))
     _check(inp, run_prefill(inp), BF16_TOL)
 
 
