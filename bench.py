@@ -52,7 +52,8 @@ DEFAULT_WORKLOAD = "decode_long_rope"
 DEFAULT_PREFILL = "prefill_b4_s4096"
 WORKLOAD_NAMES = ["decode_b32", "decode_long_rope", "decode_paged_head", "prefill_b4_s4096",
                   "prefill_b1_s4096_h16", "tiny_prefill_f32", "decode_long_rope_qc", "prefill_b4_s4096_qc",
-                  "decode_paged_head_top8", "decode_long_rope_top32", "decode_long_rope_b2"]
+                  "decode_paged_head_top8", "decode_long_rope_top32", "decode_long_rope_b2", "decode_b32_fp8",
+                  "decode_paged_head_fp8"]
 # Denominators used when no measured peaks file is present: a B200's HBM copy
 # bandwidth (GB/s), its dense bf16 GEMM throughput as a short burst, and the
 # same GEMM held for seconds under the 1 kW power cap (TFLOP/s).
@@ -196,6 +197,11 @@ class ClockSampler:
 # workload accounting
 # ---------------------------------------------------------------------------
 
+def cache_elem_bytes(w):
+    """Bytes per cached element: 1 for an FP8 latent cache, else the dtype's."""
+    return 1 if w.cache_fp8 else (2 if w.dtype == "bf16" else 4)
+
+
 def prefill_flops(w, lengths):
     """Explicit-form algorithmic FLOPs of one prefill step, per kernel."""
     T = int(sum(lengths))
@@ -221,8 +227,9 @@ def config_dict(w, inp):
                 + (", paged (page 64)" if w.paged else "")
                 + f", {w.gate_mode} gate, lengths {w.len_law}[{w.len_lo},{w.len_hi}]"
                 + (f", low-rank query d_cq {w.d_cq}" if w.d_cq else "")
-                + (f", top-{w.gate_topk} of {w.n_heads} heads" if w.gate_mode == "head_topk" else "") + ", seed 0")
-        extra = {"sum_len": int(lens.sum()), "latent_bytes_per_step": int(lens.sum()) * w.row * 2}
+                + (f", top-{w.gate_topk} of {w.n_heads} heads" if w.gate_mode == "head_topk" else "")
+                + (f", FP8 E4M3 cache (scale {w.cache_scale})" if w.cache_fp8 else "") + ", seed 0")
+        extra = {"sum_len": int(lens.sum()), "latent_bytes_per_step": int(lens.sum()) * w.row * cache_elem_bytes(w)}
     else:
         desc = (f"{w.name}: batch {w.batch} x {w.seq_len} causal prefill, d_model {w.d_model}, H {w.n_heads}, "
                 f"d_h {w.d_h}, d_c {w.d_c}, " + (f"RoPE {w.d_rope}" if w.d_rope else "NoPE")
@@ -268,7 +275,7 @@ def oracle_sample(inp, seconds: float, start: int = 0):
             for h0 in range(0, w.n_heads, hc):
                 heads = list(range(h0, min(w.n_heads, h0 + hc)))
                 oracle.decode(p, inp["x"], inp["past"], seqs=[seq], heads=heads)
-                nbytes += int(inp["lengths"][seq]) * w.row * 2 * len(heads) / w.n_heads
+                nbytes += int(inp["lengths"][seq]) * w.row * cache_elem_bytes(w) * len(heads) / w.n_heads
                 units += 1
                 if time.perf_counter() - t0 >= seconds:
                     break
@@ -368,7 +375,7 @@ class DecodeRunner:
         self.g = torch.empty(B, w.gate_width, dtype=torch.float32, device=dev)
         self.o = torch.empty(B, w.n_heads * w.d_h, dtype=torch.bfloat16, device=dev)
         self.y = torch.empty(B, w.d_model, dtype=torch.bfloat16, device=dev)
-        self.work = float(inp["lengths"].sum()) * w.row * 2          # latent bytes per step
+        self.work = float(inp["lengths"].sum()) * w.row * cache_elem_bytes(w)   # latent bytes per step
         self.dominant = "decode_attn"
         self.kernel_work = {"decode_attn": self.work}
         # host copies for the end-to-end leg

@@ -21,6 +21,8 @@ GMLA_ERR_DEVICE_RANGE = 6
 
 GMLA_BF16 = 0
 GMLA_FP32 = 1
+GMLA_CACHE_SAME = 0
+GMLA_CACHE_FP8_E4M3 = 1
 GMLA_GATE_CHANNEL = 0
 GMLA_GATE_HEAD = 1
 GMLA_GATE_HEAD_TOPK = 2
@@ -42,6 +44,8 @@ class gmla_config(ctypes.Structure):
         ("dtype", ctypes.c_int32),
         ("d_cq", ctypes.c_int32),
         ("gate_topk", ctypes.c_int32),
+        ("cache_dtype", ctypes.c_int32),
+        ("cache_scale", ctypes.c_float),
     ]
 
 

@@ -61,7 +61,8 @@ class GatedMLA:
     def __init__(self, *, d_model: int, n_heads: int, d_h: int, d_c: int, d_rope: int = 0,
                  gate_mode: str = "channel", softmax_scale: Optional[float] = None,
                  rope_base: float = 10000.0, dtype: torch.dtype = torch.bfloat16,
-                 weights: dict, d_cq: int = 0, gate_topk: int = 0):
+                 weights: dict, d_cq: int = 0, gate_topk: int = 0, cache_fp8: bool = False,
+                 cache_scale: float = 1.0):
         self.dtype = dtype
         self.cfg = L.gmla_config()
         self.cfg.d_model, self.cfg.n_heads, self.cfg.d_h, self.cfg.d_c, self.cfg.d_rope = (
@@ -73,6 +74,8 @@ class GatedMLA:
         self.cfg.rope_base = rope_base
         self.cfg.dtype = _DT[dtype]
         self.cfg.d_cq = d_cq
+        self.cfg.cache_dtype = L.GMLA_CACHE_FP8_E4M3 if cache_fp8 else L.GMLA_CACHE_SAME
+        self.cfg.cache_scale = cache_scale
         self.weights = dict(weights)
         self.w = L.gmla_weights()
         for k in ("W_c", "W_kr", "W_q", "W_qr", "W_k", "W_v", "W_g", "b_g", "W_o", "W_dq", "W_uq"):

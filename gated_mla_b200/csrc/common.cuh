@@ -2,6 +2,7 @@
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -105,6 +106,8 @@ struct EpiSeg {
   int32_t block_stride;
   int32_t col_offset;
   int32_t out_f32;       // 1: fp32 output, 0: bf16 output
+  int32_t out_fp8;       // 1: FP8 E4M3 output of v * out_scale (an FP8 latent cache)
+  float out_scale;
   int32_t rope;
   int32_t cache_scatter;
   // optional gate: v *= sigmoid(gate[t * gate_stride + f / gate_div]), or with
@@ -163,6 +166,18 @@ static __device__ __noinline__ float rope_rotate(float v, float partner, bool od
   return odd ? (partner * s + v * c) : (v * c - partner * s);
 }
 
+// One output element of an epilogue in the segment's format: fp32, bf16, or an
+// FP8 E4M3 code of v * out_scale (round to nearest even, saturating).
+__device__ __forceinline__ void store_out(const EpiSeg& e, int64_t off, float v) {
+  if (e.out_f32)
+    static_cast<float*>(e.out)[off] = v;
+  else if (e.out_fp8)
+    static_cast<uint8_t*>(e.out)[off] =
+        static_cast<uint8_t>(__nv_cvt_float_to_fp8(v * e.out_scale, __NV_SATFINITE, __NV_E4M3));
+  else
+    static_cast<__nv_bfloat16*>(e.out)[off] = __float2bfloat16_rn(v);
+}
+
 __device__ __forceinline__ void epi_store(const EpiSeg& e, int64_t row, int f, float v, int t = 0) {
   if (e.gate) {
     const float g = e.gate[static_cast<int64_t>(t) * e.gate_stride + f / e.gate_div];
@@ -171,10 +186,7 @@ __device__ __forceinline__ void epi_store(const EpiSeg& e, int64_t row, int f, f
   const int64_t off = row * e.row_stride + static_cast<int64_t>(f / e.block) * e.block_stride + (f % e.block) +
                       e.col_offset;
   if (e.bias) v += e.bias[f];
-  if (e.out_f32)
-    static_cast<float*>(e.out)[off] = v;
-  else
-    static_cast<__nv_bfloat16*>(e.out)[off] = __float2bfloat16_rn(v);
+  store_out(e, off, v);
 }
 
 }  // namespace gmla

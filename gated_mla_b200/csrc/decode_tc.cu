@@ -852,15 +852,22 @@ cudaError_t launch_decode_merge_ranks(const MergeRanksArgs& a, cudaStream_t st) 
   return e;
 }
 
+}  // namespace gmla
+
+#include "decode_fp8.cuh"
+
+namespace gmla {
+
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-DecodeLayout decode_layout(int B, int H, int eff_heads, int d_h, int d_c, int d_rope, int num_sms) {
+DecodeLayout decode_layout(int B, int H, int eff_heads, int d_h, int d_c, int d_rope, int num_sms, bool fp8) {
   DecodeLayout L{};
   const int E = eff_heads;
   L.HG = E <= 16 ? 16 : (E % 64 == 0 ? 64 : (E % 32 == 0 ? 32 : 16));
+  if (fp8 && L.HG > 32) L.HG = 32;   // hi and lo columns of 64 heads would not fit tensor memory
   L.n_hg = (E + L.HG - 1) / L.HG;
   L.G = num_sms / L.n_hg;
   if (L.G < 1) L.G = 1;
@@ -868,7 +875,11 @@ DecodeLayout decode_layout(int B, int H, int eff_heads, int d_h, int d_c, int d_
   const size_t row = static_cast<size_t>(d_c + d_rope);
   size_t off = 256;   // status word
   L.off_qa = off;
-  off = align256(off + static_cast<size_t>(B) * H * row * 2 + 16 * row * 2 /* padded head rows */);
+  {
+    const size_t bf16_q = static_cast<size_t>(B) * H * row * 2 + 16 * row * 2;   // + padded head rows
+    const size_t fp8_q = static_cast<size_t>(B) * ((H + L.HG - 1) / L.HG) * 2 * L.HG * d_c;
+    off = align256(off + (fp8 ? (fp8_q > bf16_q ? fp8_q : bf16_q) : bf16_q));
+  }
   L.off_opart = off;
   off = align256(off + static_cast<size_t>(L.n_hg) * L.max_seg * L.HG * kDc * 4);
   L.off_ml = off;
@@ -890,6 +901,8 @@ DecodeLayout decode_layout(int B, int H, int eff_heads, int d_h, int d_c, int d_
   off = align256(off + static_cast<size_t>(B) * H * 4);
   L.off_nact = off;
   off = align256(off + static_cast<size_t>(B) * 4);
+  L.off_qmul = off;
+  off = align256(off + static_cast<size_t>(B) * H * 4);
   L.total = off;
   return L;
 }
@@ -906,7 +919,26 @@ static cudaError_t launch_attn(const DecodeArgs& a, cudaStream_t st) {
   return e;
 }
 
+static cudaError_t launch_decode_fp8(DecodeArgs& a, cudaStream_t st) {
+  const int n_absorb = a.H * ((a.B + kAbs8B - 1) / kAbs8B);
+  prof_begin(st, "decode_absorb_plan");
+  cudaError_t e = launch_pdl(decode_absorb_fp8_kernel, dim3(n_absorb + 1), dim3(256), 0, st, 1, a);
+  prof_end(st);
+  if (e != cudaSuccess) return e;
+  switch (a.HG) {
+    case 16: e = launch_attn_fp8<16>(a, st); break;
+    case 32: e = launch_attn_fp8<32>(a, st); break;
+    default: return cudaErrorInvalidValue;
+  }
+  if (e != cudaSuccess) return e;
+  prof_begin(st, "decode_merge");
+  e = launch_pdl(decode_merge_kernel, dim3(a.H, a.B), dim3(128), 0, st, 1, a);
+  prof_end(st);
+  return e;
+}
+
 cudaError_t launch_decode_bf16(DecodeArgs& a, cudaStream_t st) {
+  if (a.fp8) return launch_decode_fp8(a, st);
   const int n_absorb = a.H * ((a.B + kAbsorbB - 1) / kAbsorbB) * (a.d_c / kAbsorbCols);
   prof_begin(st, "decode_absorb_plan");
   cudaError_t e = launch_pdl(decode_absorb_plan_kernel, dim3(n_absorb + 1), dim3(256), 0, st, 1, a);

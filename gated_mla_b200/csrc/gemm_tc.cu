@@ -305,10 +305,7 @@ __global__ void __launch_bounds__(192, kSwap ? 1 : 2) gemm_bf16_tc_kernel(const 
             val += fbias;
             if (e.gate) val *= e.gate_value ? gl[j] : __fdividef(1.f, 1.f + __expf(-gl[j]));
             const int64_t off = row * e.row_stride + colpart;
-            if (e.out_f32)
-              static_cast<float*>(e.out)[off] = val;
-            else
-              static_cast<__nv_bfloat16*>(e.out)[off] = __float2bfloat16_rn(val);
+            store_out(e, off, val);
           }
         };
         if (!split) {
@@ -357,7 +354,7 @@ __global__ void __launch_bounds__(192, kSwap ? 1 : 2) gemm_bf16_tc_kernel(const 
           const int64_t off16 = row * e.row_stride + static_cast<int64_t>(f0 / e.block) * e.block_stride +
                                 (f0 % e.block) + e.col_offset;
           const bool whole = !e.gate && (f0 + 16 <= seg_rows) && (f0 % e.block) + 16 <= e.block;
-          const bool vec = whole && !e.out_f32 && !e.bias && off16 % 8 == 0;
+          const bool vec = whole && !e.out_f32 && !e.out_fp8 && !e.bias && off16 % 8 == 0;
           const bool vec32 = whole && e.out_f32 && off16 % 4 == 0;   // fp32 rows (+ bias), 16-byte stores
           if (vec32) {
             float4* dst = reinterpret_cast<float4*>(static_cast<float*>(e.out) + off16);
@@ -491,10 +488,7 @@ __global__ void __launch_bounds__(192, kSwap ? 1 : 2) gemm_bf16_tc_kernel(const 
             val += fbias;
             if (e.gate) val *= e.gate_value ? gl[j] : __fdividef(1.f, 1.f + __expf(-gl[j]));
             const int64_t off = row * e.row_stride + colpart;
-            if (e.out_f32)
-              static_cast<float*>(e.out)[off] = val;
-            else
-              static_cast<__nv_bfloat16*>(e.out)[off] = __float2bfloat16_rn(val);
+            store_out(e, off, val);
           }
         }
       }

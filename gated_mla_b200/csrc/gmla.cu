@@ -92,6 +92,11 @@ gmla_status check_cfg(const gmla_config* c) {
     return fail(GMLA_ERR_INVALID_ARG, "gate_mode must be one of the gmla_gate_mode values");
   if (c->gate_mode == GMLA_GATE_HEAD_TOPK && (c->gate_topk < 1 || c->gate_topk > c->n_heads))
     return fail(GMLA_ERR_INVALID_ARG, "gate_topk must be in [1, n_heads] for GMLA_GATE_HEAD_TOPK");
+  if (c->cache_dtype != GMLA_CACHE_SAME && c->cache_dtype != GMLA_CACHE_FP8_E4M3)
+    return fail(GMLA_ERR_INVALID_ARG, "cache_dtype must be a gmla_cache_dtype value");
+  if (c->cache_dtype == GMLA_CACHE_FP8_E4M3 &&
+      (c->dtype != GMLA_BF16 || !(c->cache_scale > 0.f) || !std::isfinite(c->cache_scale)))
+    return fail(GMLA_ERR_INVALID_ARG, "an FP8 cache needs the bf16 dtype and a finite cache_scale > 0");
   if (c->dtype != GMLA_BF16 && c->dtype != GMLA_FP32) return fail(GMLA_ERR_INVALID_ARG, "dtype");
   if (!(c->softmax_scale > 0.f) || !std::isfinite(c->softmax_scale))
     return fail(GMLA_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
@@ -108,6 +113,10 @@ bool cfg_valid(const gmla_config* c) {
   if (c->d_rope % 2) return false;
   if (c->gate_mode < GMLA_GATE_CHANNEL || c->gate_mode > GMLA_GATE_HEAD_TERNARY) return false;
   if (c->gate_mode == GMLA_GATE_HEAD_TOPK && (c->gate_topk < 1 || c->gate_topk > c->n_heads)) return false;
+  if (c->cache_dtype != GMLA_CACHE_SAME && c->cache_dtype != GMLA_CACHE_FP8_E4M3) return false;
+  if (c->cache_dtype == GMLA_CACHE_FP8_E4M3 &&
+      (c->dtype != GMLA_BF16 || !(c->cache_scale > 0.f) || !std::isfinite(c->cache_scale)))
+    return false;
   if (c->dtype != GMLA_BF16 && c->dtype != GMLA_FP32) return false;
   if (!(c->softmax_scale > 0.f) || !std::isfinite(c->softmax_scale)) return false;
   if (c->d_rope && !(c->rope_base > 1.f)) return false;
@@ -256,6 +265,33 @@ bool make_tmap_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t d1,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool make_tmap_2d_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t row_stride_bytes,
+                     uint32_t box_inner, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {row_stride_bytes};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_tmap_3d_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t d1, uint64_t d2,
+                     uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box_inner, uint32_t box1,
+                     uint32_t box2) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {inner, d1, d2};
+  cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
+  cuuint32_t box[3] = {box_inner, box1, box2};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace gmla
 
 // ===========================================================================
@@ -322,7 +358,8 @@ size_t gmla_gate_out_workspace_size(const gmla_config* cfg, int32_t T) {
 size_t gmla_decode_workspace_size(const gmla_config* cfg, int32_t B) {
   if (!cfg_valid(cfg) || B < 0) return 256;
   if (cfg->dtype == GMLA_FP32) return 256;
-  return decode_layout(B, cfg->n_heads, decode_eff_heads(cfg), cfg->d_h, cfg->d_c, cfg->d_rope, num_sms()).total;
+  return decode_layout(B, cfg->n_heads, decode_eff_heads(cfg), cfg->d_h, cfg->d_c, cfg->d_rope, num_sms(),
+                       cfg->cache_dtype == GMLA_CACHE_FP8_E4M3).total;
 }
 
 size_t gmla_prefill_workspace_size(const gmla_config* cfg, int32_t T, int32_t B) {
@@ -476,8 +513,14 @@ gmla_status gmla_latent_project(const gmla_config* cfg, const gmla_weights* w, c
   const EpiSeg e_qr = plain_seg(q_out, static_cast<int64_t>(H) * dq, dr, dq, dh, f32, nullptr, true, false);
   ProjSeg segs[kMaxSeg];
   int ns = 0;
-  segs[ns++] = {w->W_c, dc, plain_seg(cache->data, row, 1 << 30, 0, 0, f32, nullptr, false, true)};
-  if (dr) segs[ns++] = {w->W_kr, dr, plain_seg(cache->data, row, dr, 0, dc, f32, nullptr, true, true)};
+  EpiSeg e_c = plain_seg(cache->data, row, 1 << 30, 0, 0, f32, nullptr, false, true);
+  EpiSeg e_kr = plain_seg(cache->data, row, dr, 0, dc, f32, nullptr, true, true);
+  if (cfg->cache_dtype == GMLA_CACHE_FP8_E4M3) {   // the cache stores E4M3 codes of value / cache_scale
+    e_c.out_fp8 = e_kr.out_fp8 = 1;
+    e_c.out_scale = e_kr.out_scale = 1.f / cfg->cache_scale;
+  }
+  segs[ns++] = {w->W_c, dc, e_c};
+  if (dr) segs[ns++] = {w->W_kr, dr, e_kr};
   if (compressed) {
     segs[ns++] = {w->W_dq, cfg->d_cq, plain_seg(cq, cfg->d_cq, 1 << 30, 0, 0, f32, nullptr, false, false)};
   } else {
@@ -557,13 +600,25 @@ static gmla_status decode_impl(const gmla_config* cfg, const gmla_weights* w, co
   if (cfg->d_c != 512 || (cfg->d_rope != 0 && cfg->d_rope != 64))
     return fail(GMLA_ERR_UNSUPPORTED, "bf16 decode covers d_c = 512 with d_rope in {0, 64}");
   if (cfg->d_h != 128 && cfg->d_h != 256) return fail(GMLA_ERR_UNSUPPORTED, "bf16 decode covers d_h in {128, 256}");
+  const bool fp8 = cfg->cache_dtype == GMLA_CACHE_FP8_E4M3;
+  if (fp8 && (cfg->d_rope != 0 || cfg->d_c != 512))
+    return fail(GMLA_ERR_UNSUPPORTED, "an FP8 cache covers NoPE decode with d_c = 512");
   const DecodeLayout L = decode_layout(B, cfg->n_heads, decode_eff_heads(cfg), cfg->d_h, cfg->d_c, cfg->d_rope,
-                                       num_sms());
+                                       num_sms(), fp8);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   DecodeArgs a{};
   const int row = cfg->d_c + cfg->d_rope;
   const int tile_rows = 128;   // tokens per attention tile
-  if (!cache->paged) {
+  if (fp8) {
+    // codes: [rows, row] bytes, boxes of 128 tokens x 128 latent dims
+    const bool okm = !cache->paged
+                         ? make_tmap_2d_u8(&a.cache_map, cache->data, row,
+                                           static_cast<uint64_t>(cache->batch) * cache->capacity, row, 128, tile_rows)
+                         : make_tmap_3d_u8(&a.cache_map, cache->data, row, cache->page_size, cache->num_pages, row,
+                                           static_cast<uint64_t>(row) * cache->page_size, 128,
+                                           cache->page_size < tile_rows ? cache->page_size : tile_rows, 1);
+    if (!okm) return fail(GMLA_ERR_CUDA, "tensor map for the FP8 cache failed");
+  } else if (!cache->paged) {
     if (!make_tmap_2d(&a.cache_map, cache->data, row, static_cast<uint64_t>(cache->batch) * cache->capacity,
                       static_cast<uint64_t>(row) * 2, 64, tile_rows, true))
       return fail(GMLA_ERR_CUDA, "tensor map for the cache failed");
@@ -573,8 +628,10 @@ static gmla_status decode_impl(const gmla_config* cfg, const gmla_weights* w, co
                       static_cast<uint64_t>(row) * 2 * ps, 64, ps < tile_rows ? ps : tile_rows, 1, true))
       return fail(GMLA_ERR_CUDA, "tensor map for the paged cache failed");
   }
-  if (!make_tmap_2d(&a.qa_map, ws + L.off_qa, row, static_cast<uint64_t>(B) * cfg->n_heads,
-                    static_cast<uint64_t>(row) * 2, 64, L.HG, true))
+  if (fp8 ? !make_tmap_2d_u8(&a.qa_map, ws + L.off_qa, cfg->d_c, static_cast<uint64_t>(B) * L.n_hg * 2 * L.HG,
+                             cfg->d_c, 128, 2 * L.HG)
+          : !make_tmap_2d(&a.qa_map, ws + L.off_qa, row, static_cast<uint64_t>(B) * cfg->n_heads,
+                          static_cast<uint64_t>(row) * 2, 64, L.HG, true))
     return fail(GMLA_ERR_CUDA, "tensor map for the absorbed queries failed");
   a.cache = cv;
   a.seq_lens = seq_lens;
@@ -609,6 +666,9 @@ static gmla_status decode_impl(const gmla_config* cfg, const gmla_weights* w, co
   a.n_act = reinterpret_cast<int32_t*>(ws + L.off_nact);
   a.seq_starts = seq_starts;
   a.partial_out = partial_out;
+  a.fp8 = fp8 ? 1 : 0;
+  a.cache_scale = cfg->cache_scale;
+  a.qmul = reinterpret_cast<float*>(ws + L.off_qmul);
   a.olat = ws + L.off_olat;
   const SwapPlan& sp = L.gemm_plan;
   a.gemm_counters = nullptr;
@@ -748,6 +808,8 @@ gmla_status gmla_prefill(const gmla_config* cfg, const gmla_weights* w, const vo
   if (B == 0 || T == 0) return GMLA_OK;
   if (B > cache->batch) return fail(GMLA_ERR_INVALID_ARG, "B (%d) exceeds cache.batch (%d)", B, cache->batch);
   if (cache->paged) return fail(GMLA_ERR_UNSUPPORTED, "prefill reads a contiguous cache");
+  if (cfg->cache_dtype == GMLA_CACHE_FP8_E4M3)
+    return fail(GMLA_ERR_UNSUPPORTED, "prefill reads a bf16 or fp32 cache (an FP8 cache is read by decode)");
   if (max_seqlen > cache->capacity) return fail(GMLA_ERR_INVALID_ARG, "max_seqlen exceeds cache.capacity");
   GMLA_TRY(check_ptr(q, "q"));
   GMLA_TRY(check_ptr(cu_seqlens, "cu_seqlens"));

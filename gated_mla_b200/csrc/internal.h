@@ -94,6 +94,11 @@ struct DecodeArgs {
   // (null: from 0), and write per-(sequence, head) partials instead of O_lat
   const int32_t* seq_starts;
   float* partial_out;        // [B, H, d_c + 4]: O_lat / l, then log2-domain m + log2 l
+  // FP8 (E4M3) latent cache: codes times cache_scale; the absorbed queries are
+  // hi/lo e4m3 rows [B, n_hg, 2, HG, d_c] with one multiplier per (sequence, slot)
+  int32_t fp8;
+  float cache_scale;
+  float* qmul;               // workspace: [B, H] sigma * cache_scale
 };
 
 // Cross-rank merge of context-parallel partials into O_lat (bf16 [H, B, d_c]),
@@ -111,13 +116,13 @@ constexpr int kPartialPad = 4;   // floats after the d_c values of a partial row
 
 struct DecodeLayout {
   size_t off_qa, off_opart, off_ml, off_seg, off_seqfirst, off_ctafirst, off_olat, off_gemm;
-  size_t off_gvals, off_hslot, off_nact, total;
+  size_t off_gvals, off_hslot, off_nact, off_qmul, total;
   int HG, n_hg, G, max_seg;
   SwapPlan gemm_plan;        // the W_v GEMM (heads x 128 rows, B tokens, K = d_c)
 };
 // eff_heads: the most heads a sequence attends with (H, or k with top-k gates),
 // which sets the head groups of the attention kernel.
-DecodeLayout decode_layout(int B, int H, int eff_heads, int d_h, int d_c, int d_rope, int num_sms);
+DecodeLayout decode_layout(int B, int H, int eff_heads, int d_h, int d_c, int d_rope, int num_sms, bool fp8 = false);
 cudaError_t launch_decode_bf16(DecodeArgs& a, cudaStream_t st);
 
 // ----- fp32 CUDA-core path (simt_f32.cu) -----
@@ -189,5 +194,11 @@ bool make_tmap_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t row
 bool make_tmap_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t d1, uint64_t d2,
                   uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box_inner, uint32_t box1,
                   uint32_t box2, bool swizzle128);
+// the same over one-byte elements (FP8 codes)
+bool make_tmap_2d_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t row_stride_bytes,
+                     uint32_t box_inner, uint32_t box_rows);
+bool make_tmap_3d_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t d1, uint64_t d2,
+                     uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box_inner, uint32_t box1,
+                     uint32_t box2);
 
 }  // namespace gmla

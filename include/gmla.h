@@ -73,6 +73,16 @@ typedef enum gmla_status {
 
 typedef enum gmla_dtype { GMLA_BF16 = 0, GMLA_FP32 = 1 } gmla_dtype;
 
+/* Latent cache element format. GMLA_CACHE_SAME: the config's dtype.
+ * GMLA_CACHE_FP8_E4M3: one byte per element, an E4M3 code (round to nearest
+ * even, saturating at +-448) of value / cache_scale, one fp32 scale for the
+ * whole cache. It halves the cache bytes a decode reads; the "Kimi K3" gating
+ * blog (zwxr.cn) §7 warns that quantisation errors compound, and the library
+ * keeps every other operand near bf16 precision. bf16 dtype only: decode
+ * (NoPE, d_c = 512) reads it and gmla_latent_project writes it; gmla_prefill
+ * over an FP8 cache returns GMLA_ERR_UNSUPPORTED. */
+typedef enum gmla_cache_dtype { GMLA_CACHE_SAME = 0, GMLA_CACHE_FP8_E4M3 = 1 } gmla_cache_dtype;
+
 /* Per-channel gate: G = H*d_h ("Gated MLA 计算公式" §二 boxed equation).
  * Per-head gate:    G = H, broadcast over the head's d_h channels
  *                   ("Gated Multi-head Latent Attention", "Gating Mechanism").
@@ -107,6 +117,8 @@ typedef struct gmla_config {
   int32_t d_cq;           /* low-rank query width d_cq ("精读笔记 03" §5.1: c^Q = W^DQ h,
                              q = W^UQ c^Q; §5.2: q^R = RoPE(W^QR c^Q)); 0 = full-rank query */
   int32_t gate_topk;      /* k of GMLA_GATE_HEAD_TOPK (1 <= k <= H); ignored otherwise */
+  int32_t cache_dtype;    /* gmla_cache_dtype: the latent cache's element format */
+  float cache_scale;      /* GMLA_CACHE_FP8_E4M3: a stored code e means cache_scale * e */
 } gmla_config;
 
 typedef struct gmla_weights {

@@ -47,7 +47,7 @@ from typing import Optional, Sequence
 import numpy as np
 
 __all__ = [
-    "params", "sigmoid", "rope", "latent", "project", "project_latent", "project_query", "head_kv",
+    "params", "sigmoid", "rope", "round_e4m3", "cache_store", "latent", "project", "project_latent", "project_query", "head_kv",
     "attention_explicit", "attention_absorbed", "head_gate_values", "gate", "output",
     "prefill", "decode", "kv_elements_per_token", "kv_bytes_per_token",
 ]
@@ -72,6 +72,7 @@ def params(inputs: dict) -> dict:
     return {
         "H": w.n_heads, "d_h": w.d_h, "d_c": w.d_c, "d_R": w.d_rope,
         "d_model": w.d_model, "gate_mode": w.gate_mode, "gate_topk": w.gate_topk,
+        "cache_fp8": w.cache_fp8, "cache_scale": w.cache_scale,
         "scale": w.softmax_scale, "rope_base": w.rope_base,
         "W_c": f(inputs["W_c"]), "W_kr": f(inputs.get("W_kr")),
         "W_q": f(inputs.get("W_q")), "W_qr": f(inputs.get("W_qr")),
@@ -118,6 +119,34 @@ def rope(v: np.ndarray, pos: np.ndarray, base: float) -> np.ndarray:
     return out
 
 
+E4M3_MAX = 448.0
+
+
+def round_e4m3(v: np.ndarray) -> np.ndarray:
+    """Nearest FP8 E4M3 value (1 sign, 4 exponent bits with bias 7, 3 mantissa
+    bits; subnormals below 2^-6 in steps of 2^-9; largest finite 448), ties to
+    the even code, saturating to +-448. Values are returned as float64."""
+    v = np.asarray(v, dtype=np.float64)
+    a = np.abs(v)
+    _, e = np.frexp(a)                        # a = f * 2^e, f in [0.5, 1)
+    ulp = np.ldexp(1.0, np.maximum(e - 1, -6) - 3)   # 3 mantissa bits; subnormal step 2^-9
+    q = np.round(a / ulp) * ulp               # numpy rounds halves to even
+    q = np.minimum(q, E4M3_MAX)
+    return np.copysign(q, v)
+
+
+def cache_store(p: dict, row: np.ndarray) -> np.ndarray:
+    """The value a cached element holds: itself in a bf16/fp32 cache; with an
+    FP8 latent cache, cache_scale * e4m3(row / cache_scale) (reading: one fp32
+    scale for the whole cache, codes rounded to nearest even and saturated;
+    the [K3 blog] §7 warns that such quantisation errors compound, so the
+    oracle models the stored value exactly)."""
+    if not p.get("cache_fp8"):
+        return row
+    s = p["cache_scale"]
+    return s * round_e4m3(np.asarray(row, np.float64) / s)
+
+
 def latent(W_c: np.ndarray, x: np.ndarray) -> np.ndarray:
     """c_s = W_c x_s ([MLA-gate] §一; [MLA-notes] §5.1 c^KV = W^DKV h). x [T, d_model]."""
     return x @ W_c.T
@@ -128,11 +157,14 @@ def project_latent(p: dict, x: np.ndarray, positions: np.ndarray) -> dict:
 
     * c  [T, d_c]   latent c = W_c x
     * kR [T, d_R]   RoPE(W_kr x) at the token's position (shared by all heads)
+
+    Both are returned as the cache stores them (cache_store: rounded to FP8
+    E4M3 times the cache scale for an FP8 latent cache).
     """
     x = np.asarray(x, dtype=np.float64)
-    out = {"c": latent(p["W_c"], x)}
+    out = {"c": cache_store(p, latent(p["W_c"], x))}
     if p["d_R"]:
-        out["kR"] = rope(x @ p["W_kr"].T, positions, p["rope_base"])
+        out["kR"] = cache_store(p, rope(x @ p["W_kr"].T, positions, p["rope_base"]))
     else:
         out["kR"] = np.zeros((x.shape[0], 0))
     return out

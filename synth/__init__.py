@@ -25,6 +25,8 @@ Workloads (sizes as named in the problem statement of Gated MLA):
 * ``decode_long_rope_qc``, ``prefill_b4_s4096_qc``: the long-context decode
                          and the batch-4 prefill with a low-rank query,
                          d_cq 1536.
+* ``decode_b32_fp8``, ``decode_paged_head_fp8``: the batch-32 and the paged decode
+                         over an FP8 E4M3 latent cache (one scale, 1/64).
 * ``decode_paged_head_top8``, ``decode_long_rope_top32``: the paged decode and
                          the long-context decode with hard top-k per-head
                          gates (8 of 32, 32 of 128 heads).
@@ -41,7 +43,7 @@ from typing import Optional
 
 import numpy as np
 
-__all__ = ["Workload", "WORKLOADS", "workload", "generate", "bf16_round",
+__all__ = ["Workload", "WORKLOADS", "workload", "generate", "bf16_round", "e4m3_round",
            "bf16_bits", "bits_to_f32"]
 
 
@@ -68,6 +70,8 @@ class Workload:
     paged: bool = False
     page_size: int = 64
     d_cq: int = 0           # query low-rank compression width; 0 = full-rank query
+    cache_fp8: bool = False  # FP8 E4M3 latent cache with one fp32 scale
+    cache_scale: float = 1.0 / 64.0
 
     @property
     def softmax_scale(self) -> float:
@@ -132,6 +136,14 @@ WORKLOADS = {
         name="decode_long_rope_top32", mode="decode", dtype="bf16", batch=8, d_model=7168,
         n_heads=128, d_h=128, d_c=512, d_rope=64, rope_base=10000.0, gate_mode="head_topk", gate_topk=32,
         gate_bias=True, len_law="fixed", len_lo=131072, len_hi=131072),
+    # the batch-32 and the paged decode over an FP8 (E4M3) latent cache, scale 1/64
+    "decode_b32_fp8": Workload(
+        name="decode_b32_fp8", mode="decode", dtype="bf16", batch=32, d_model=2048,
+        n_heads=16, d_h=128, d_c=512, len_law="uniform", len_lo=1024, len_hi=8192, cache_fp8=True),
+    "decode_paged_head_fp8": Workload(
+        name="decode_paged_head_fp8", mode="decode", dtype="bf16", batch=64, d_model=4096,
+        n_heads=32, d_h=128, d_c=512, gate_mode="head", gate_bias=True,
+        len_law="loguniform", len_lo=256, len_hi=32768, paged=True, page_size=64, cache_fp8=True),
     "prefill_b4_s4096_qc": Workload(
         name="prefill_b4_s4096_qc", mode="prefill", dtype="bf16", batch=4, seq_len=4096,
         d_model=7168, n_heads=64, d_h=128, d_c=512, gate_bias=True, d_cq=1536),
@@ -163,6 +175,14 @@ def bf16_bits(a: np.ndarray) -> np.ndarray:
 def bits_to_f32(b: np.ndarray) -> np.ndarray:
     """bfloat16 bit patterns (uint16) -> float32 (exact)."""
     return (np.ascontiguousarray(b, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+def e4m3_round(a: np.ndarray) -> np.ndarray:
+    """float32 values rounded to the nearest FP8 E4M3 value (ties to even,
+    saturating at +-448), kept as float32: torch's float8 conversion."""
+    import torch
+    t = torch.from_numpy(np.clip(np.ascontiguousarray(a, dtype=np.float32), -448.0, 448.0))
+    return t.to(torch.float8_e4m3fn).to(torch.float32).numpy()
 
 
 def bf16_round(a: np.ndarray) -> np.ndarray:
@@ -261,6 +281,11 @@ def generate(w: Workload, seed: int = 0, lengths: Optional[np.ndarray] = None) -
         if w.paged:
             n_pages = int(sum((int(L) + w.page_size - 1) // w.page_size for L in lens))
             out["page_perm"] = rng.permutation(n_pages).astype(np.int64)
-        out["past"] = [rnd(_normal(rng, (int(L) - 1, w.row), 1.0)) if L > 1
+        if w.cache_fp8:   # stored values: scale * an E4M3 code
+            sc = np.float32(w.cache_scale)
+            cache_rnd = lambda a: e4m3_round(a / sc) * sc
+        else:
+            cache_rnd = rnd
+        out["past"] = [cache_rnd(_normal(rng, (int(L) - 1, w.row), 1.0)) if L > 1
                        else np.zeros((0, w.row), np.float32) for L in lens]
     return out

@@ -46,7 +46,15 @@ def make_model(inp, device="cuda"):
     weights["b_g"] = dev(inp["b_g"], torch.float32)
     return GatedMLA(d_model=w.d_model, n_heads=w.n_heads, d_h=w.d_h, d_c=w.d_c, d_rope=w.d_rope,
                     gate_mode=w.gate_mode, softmax_scale=w.softmax_scale, rope_base=w.rope_base,
-                    dtype=dt, weights=weights, d_cq=w.d_cq, gate_topk=w.gate_topk)
+                    dtype=dt, weights=weights, d_cq=w.d_cq, gate_topk=w.gate_topk, cache_fp8=w.cache_fp8,
+                    cache_scale=w.cache_scale)
+
+
+def _filled(shape, fill, dt, device):
+    if dt == torch.float8_e4m3fn:   # NaN is the code 0x7f, zero the code 0x00
+        code = 0x7F if fill != fill else 0x00
+        return torch.full(shape, code, dtype=torch.uint8, device=device).view(torch.float8_e4m3fn)
+    return torch.full(shape, fill, dtype=dt, device=device)
 
 
 def make_decode_cache(inp, device="cuda", paged=None, capacity=None, fill=float("nan")):
@@ -57,9 +65,13 @@ def make_decode_cache(inp, device="cuda", paged=None, capacity=None, fill=float(
     lens = [int(L) for L in inp["lengths"]]
     B = w.batch
     paged = w.paged if paged is None else paged
+    if w.cache_fp8:   # E4M3 codes of the stored values / cache_scale (exact: the values are on the grid)
+        dt = torch.float8_e4m3fn
+        scale = np.float32(w.cache_scale)
+        inp = dict(inp, past=[r / scale for r in inp["past"]])
     if not paged:
         cap = capacity or max(1, max(lens))
-        data = torch.full((B, cap, w.row), fill, dtype=dt, device=device)
+        data = _filled((B, cap, w.row), fill, dt, device)
         for b, rows in enumerate(inp["past"]):
             if len(rows):
                 data[b, :len(rows)] = torch.from_numpy(rows).to(device, dt)
@@ -72,7 +84,7 @@ def make_decode_cache(inp, device="cuda", paged=None, capacity=None, fill=float(
         perm = np.random.default_rng(7).permutation(total)
     mpps = max(npg)
     bt = np.full((B, mpps), -1, dtype=np.int32)
-    data = torch.full((total, ps, w.row), fill, dtype=dt, device=device)
+    data = _filled((total, ps, w.row), fill, dt, device)
     k = 0
     for b in range(B):
         for p in range(npg[b]):

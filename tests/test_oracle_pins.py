@@ -675,3 +675,68 @@ def test_peaked_decode_input_needs_the_rescale():
             bad = _online_latent(z[h], C, rescale=False)
             worst = max(worst, np.linalg.norm(bad - exact) / np.linalg.norm(exact))
     assert worst > 1.0, worst
+
+
+# ---------------------------------------------------------------------------
+# FP8 latent cache: the stored value is cache_scale * e4m3(c / cache_scale)
+# ---------------------------------------------------------------------------
+
+def _e4m3_table():
+    """Every finite E4M3 value, decoded from its bits by the format's
+    definition: sign, 4 exponent bits (bias 7), 3 mantissa bits, subnormals at
+    exponent 0, and the all-ones code (S.1111.111) left out as NaN."""
+    vals = []
+    for code in range(256):
+        s, e, m = code >> 7, (code >> 3) & 15, code & 7
+        if e == 15 and m == 7:
+            continue
+        mag = (m / 8.0) * 2.0 ** -6 if e == 0 else (1.0 + m / 8.0) * 2.0 ** (e - 7)
+        vals.append(-mag if s else mag)
+    return np.array(sorted(set(vals)))
+
+
+def test_e4m3_rounding_matches_the_format_definition():
+    table = _e4m3_table()
+    assert table.max() == 448.0 and np.min(np.abs(table[table != 0])) == 2.0 ** -9
+    np.testing.assert_array_equal(oracle.round_e4m3(table), table)      # representable values are fixed
+    # midpoints between neighbours go to the even code; positive magnitudes in
+    # increasing order are the codes 0x00, 0x01, ... so a code's parity is its index's
+    pos = table[table >= 0]
+    mids = (pos[1:] + pos[:-1]) / 2
+    got = oracle.round_e4m3(mids)
+    want = np.where(np.arange(len(mids)) % 2 == 0, pos[:-1], pos[1:])
+    np.testing.assert_array_equal(got, want)
+    np.testing.assert_array_equal(oracle.round_e4m3(-mids), -want)
+    assert oracle.round_e4m3(np.array([500.0, -1e9]))[0] == 448.0 and oracle.round_e4m3(np.array([-1e9]))[0] == -448.0
+    rng = np.random.default_rng(0)
+    x = rng.standard_normal(100000) * 50
+    q = oracle.round_e4m3(x)
+    # the nearest representable value: no table entry is closer
+    idx = np.searchsorted(table, x)
+    lo = table[np.clip(idx - 1, 0, len(table) - 1)]
+    hi = table[np.clip(idx, 0, len(table) - 1)]
+    assert np.all(np.abs(q - x) <= np.minimum(np.abs(lo - x), np.abs(hi - x)) + 1e-12)
+
+
+def test_e4m3_rounding_agrees_with_torch_float8():
+    import torch
+    x = np.random.default_rng(1).standard_normal(200000).astype(np.float32) * 40
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    np.testing.assert_array_equal(oracle.round_e4m3(x), ref)
+
+
+def test_fp8_cache_rows_and_their_error_bound():
+    w = synth.Workload(name="f8", mode="decode", dtype="bf16", batch=2, d_model=16, n_heads=2, d_h=4, d_c=8,
+                       cache_fp8=True, cache_scale=1 / 32)
+    inp = synth.generate(w, seed=0, lengths=np.array([5, 9]))
+    p = oracle.params(inp)
+    for rows in inp["past"]:                                             # past rows are already stored values
+        np.testing.assert_array_equal(oracle.cache_store(p, rows.astype(np.float64)), rows)
+    c = oracle.latent(p["W_c"], np.asarray(inp["x"], float))
+    stored = oracle.project_latent(p, inp["x"], np.array([4, 8]))["c"]
+    s = p["cache_scale"]
+    assert np.all(np.abs(stored - c) <= 2.0 ** -4 * np.abs(c) + 2.0 ** -10 * s)
+    codes = stored / s
+    np.testing.assert_array_equal(oracle.round_e4m3(codes), codes)
+    # a bf16 cache stores values as they are
+    assert oracle.cache_store(dict(p, cache_fp8=False), c) is c
