@@ -79,6 +79,9 @@ def parse():
                     help="prefill workload measured in the same run (its own object in the line)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle CPU baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cp-shares", type=int, default=1,
+                    help="decode only: run the step as a context-parallel decode of this many position "
+                         "ranges, all on this GPU (gmla_decode_partial per range, then gmla_decode_merge)")
     return ap.parse_args()
 
 
@@ -358,7 +361,7 @@ def run_reference(args):
 # ---------------------------------------------------------------------------
 
 class DecodeRunner:
-    def __init__(self, inp, dev):
+    def __init__(self, inp, dev, cp_shares=1):
         import torch
         sys.path.insert(0, os.path.join(ROOT, "tests"))
         from gpu_pipeline import make_decode_cache, make_model
@@ -382,11 +385,25 @@ class DecodeRunner:
         self.host_in = [t.cpu().pin_memory() for t in (self.x, self.seq_lens, self.positions, self.seq_ids)]
         self.dev_in = [torch.empty_like(t) for t in (self.x, self.seq_lens, self.positions, self.seq_ids)]
         self.y_host = torch.empty(B, w.d_model, dtype=torch.bfloat16).pin_memory()
+        # context-parallel emulation: the ranges of every share, run one after another here
+        self.cp = cp_shares
+        if cp_shares > 1:
+            from gated_mla_b200 import context_parallel as cpm
+            self.cpm = cpm
+            lens = [int(n) for n in inp["lengths"]]
+            self.shares = [tuple(t.to(dev) for t in cpm.shard_table(lens, cp_shares, r)) for r in range(cp_shares)]
+            self.parts = torch.empty(cp_shares, B, w.n_heads, w.d_c + cpm.PARTIAL_PAD, dtype=torch.float32,
+                                     device=dev)
 
     def step(self):
         m = self.model
         m.latent_project(self.x, self.positions, self.seq_ids, self.cache, q_out=self.q, gate_logits=self.g)
-        m.decode(self.q, self.g, self.cache, self.seq_lens, o_out=self.o)
+        if self.cp > 1:
+            for r, (starts, ends) in enumerate(self.shares):
+                self.cpm.decode_partial(m, self.q, self.g, self.cache, starts, ends, out=self.parts[r])
+            self.cpm.decode_merge(m, self.parts, self.g, out=self.o)
+        else:
+            m.decode(self.q, self.g, self.cache, self.seq_lens, o_out=self.o)
         m.gate_out(self.o, y_out=self.y)
 
     def e2e_step(self):
@@ -452,7 +469,7 @@ def measure(name, args, world, rank, dev, dist, cpu_leg):
 
     w = synth.workload(name)
     inp = synth.generate(w, seed=0)
-    run = DecodeRunner(inp, dev) if w.mode == "decode" else PrefillRunner(inp, dev)
+    run = DecodeRunner(inp, dev, args.cp_shares) if w.mode == "decode" else PrefillRunner(inp, dev)
     scale, unit = work_unit(w)
     flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=dev)
 
@@ -584,7 +601,9 @@ def measure(name, args, world, rank, dev, dist, cpu_leg):
         "metric": DECODE_METRIC if w.mode == "decode" else PREFILL_METRIC, "value": value, "unit": unit,
         "ms_per_step": max_total_ms / K,
         "dtype": "bf16" if w.dtype == "bf16" else "f32",
-        "config": dict(config_dict(w, inp), cuda_graph=True),
+        "config": dict(config_dict(w, inp), cuda_graph=True,
+                       **({"context_parallel_shares_on_one_gpu": args.cp_shares}
+                          if w.mode == "decode" and args.cp_shares > 1 else {})),
         "roofline": roof, "kernel_ms": kernel_ms, "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": int(launches_per_step * K),

@@ -12,10 +12,10 @@
 // The other operand of each product is not an FP8 quantity of the method, so it
 // is carried as a hi + lo pair of e4m3 values (v ~ hi + lo, about 7 significant
 // bits): the absorbed query as Q~ = [hi(q_lat / sigma); lo(...)] with one scale
-// sigma per (sequence, head), and P' = 256 p as [hi; lo]. The pair doubles N,
+// sigma per (sequence, head), and P' = kPScale p as [hi; lo]. The pair doubles N,
 // which costs next to nothing at these widths (an MMA with N <= 64 is bound by
 // its A operand). Scores are (S[h] + S[HG + h]) * sigma * cache_scale; the
-// weighted sum is (O^T[h] + O^T[HG + h]) * cache_scale / 256.
+// weighted sum is (O^T[h] + O^T[HG + h]) * cache_scale / kPScale.
 //
 // Kernels: decode_absorb_fp8 (q_lat, its scale and hi/lo codes; its last block
 // builds the split plan as decode_absorb_plan does), decode_attn_fp8 (below),
@@ -30,7 +30,12 @@ constexpr int kTok = 128;                  // tokens per tile
 constexpr int kBox8 = 128 * 128;           // one box: 128 token rows x 128 e4m3 latent dims
 constexpr int kNB8 = 4;                    // boxes per tile (d_c = 512)
 constexpr int kDc8 = 512;
-constexpr float kPScale = 256.f;           // P' = 256 p keeps small weights above the e4m3 subnormals
+// The running max of a head is raised only when a tile's max exceeds it by
+// more than kRaise8 (log2 units), so p = 2^(s - m) <= 2^kRaise8 and
+// P' = kPScale p <= 256, inside E4M3's range (448); weights down to
+// 2^-15 stay representable.
+constexpr float kRaise8 = 2.f;
+constexpr float kPScale = 64.f;
 
 __device__ __forceinline__ uint8_t to_e4m3(float v) {
   return static_cast<uint8_t>(__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3));
@@ -102,13 +107,23 @@ __global__ void __launch_bounds__(256) decode_absorb_fp8_kernel(DecodeArgs a) {
   float acc[kAbs8B][2];
 #pragma unroll
   for (int bi = 0; bi < kAbs8B; ++bi) acc[bi][0] = acc[bi][1] = 0.f;
-  for (int k = 0; k < a.d_h; ++k) {
-    const __nv_bfloat162 w2 = *reinterpret_cast<const __nv_bfloat162*>(Wk + static_cast<int64_t>(k) * kDc8 + c0);
-    const float w0 = __low2float(w2), w1 = __high2float(w2);
+  // 16 rows of W_k in flight at a time (the loads, not the FMAs, set the pace)
+  constexpr int kRows = 16;
+  for (int k0 = 0; k0 < a.d_h; k0 += kRows) {
+    __nv_bfloat162 w2[kRows];
 #pragma unroll
-    for (int bi = 0; bi < kAbs8B; ++bi) {
-      acc[bi][0] = fmaf(sq[bi][k], w0, acc[bi][0]);
-      acc[bi][1] = fmaf(sq[bi][k], w1, acc[bi][1]);
+    for (int i = 0; i < kRows; ++i)
+      w2[i] = k0 + i < a.d_h ? *reinterpret_cast<const __nv_bfloat162*>(Wk + static_cast<int64_t>(k0 + i) * kDc8 + c0)
+                             : __floats2bfloat162_rn(0.f, 0.f);
+#pragma unroll
+    for (int i = 0; i < kRows; ++i) {
+      if (k0 + i >= a.d_h) break;
+      const float w0 = __low2float(w2[i]), w1 = __high2float(w2[i]);
+#pragma unroll
+      for (int bi = 0; bi < kAbs8B; ++bi) {
+        acc[bi][0] = fmaf(sq[bi][k0 + i], w0, acc[bi][0]);
+        acc[bi][1] = fmaf(sq[bi][k0 + i], w1, acc[bi][1]);
+      }
     }
   }
   // per sequence: the largest |q_lat| over the 512 dims (block reduction)
@@ -131,13 +146,15 @@ __global__ void __launch_bounds__(256) decode_absorb_fp8_kernel(DecodeArgs a) {
     const float sigma = mx > 0.f ? mx / 448.f : 1.f;
     const float inv = 1.f / sigma;
     const int b = b0 + bi, slot = s_slot[bi];
+    if (threadIdx.x == 0) a.qmul[static_cast<int64_t>(b) * a.H + slot] = sigma * a.cache_scale * s_on[bi];
+    // slots past the launched head groups (heads a top-k gate switches off) are never read
+    if (slot >= a.n_hg * a.HG) continue;
     const int64_t row_hi = (static_cast<int64_t>(b) * a.n_hg + slot / a.HG) * N2 + slot % a.HG;
     uint8_t h0, l0, h1, l1;
     split_e4m3(acc[bi][0] * inv * s_on[bi], h0, l0);
     split_e4m3(acc[bi][1] * inv * s_on[bi], h1, l1);
     *reinterpret_cast<uint16_t*>(qa + row_hi * kDc8 + c0) = static_cast<uint16_t>(h0 | (h1 << 8));
     *reinterpret_cast<uint16_t*>(qa + (row_hi + a.HG) * kDc8 + c0) = static_cast<uint16_t>(l0 | (l1 << 8));
-    if (threadIdx.x == 0) a.qmul[static_cast<int64_t>(b) * a.H + slot] = sigma * a.cache_scale * s_on[bi];
   }
 }
 
@@ -155,25 +172,35 @@ struct Dec8Smem {
   float mfin[64];
 };
 
+// 16 heads per CTA: two CTAs share an SM (each holds a ring of 5 boxes, and
+// the 256 columns of tensor memory it needs), so one CTA's loads, softmax and
+// MMAs overlap the other's; each CTA on its own is bound by the latency of
+// that chain, not by bandwidth. 32 heads: one CTA per SM with a deeper ring.
 template <int HG>
 struct Dec8Cfg {
   static constexpr int kN2 = 2 * HG;                         // hi and lo columns
   static constexpr int kSG = HG >= 32 ? 2 : 1;               // softmax warp groups (head slices)
   static constexpr int kThreads = 64 + 128 * kSG;
+  static constexpr int kCtasPerSm = HG == 16 ? 2 : 1;
   static constexpr int kQBytes = kNB8 * kN2 * 128;           // 4 boxes of [2 HG rows x 128 B]
   static constexpr int kPBytes = ((kN2 * 128) + 1023) & ~1023;   // [2 HG rows x 128 tokens]
   static constexpr int kStruct = (static_cast<int>(sizeof(Dec8Smem)) + 127) & ~127;
   static constexpr int kFixed = kQBytes + kPBytes + kStruct + 1024 /*align*/;
-  static constexpr int kBudget = 232448;
+  // shared memory of an SM (233472 B) less 1 KB reserved per CTA
+  static constexpr int kBudget = kCtasPerSm == 2 ? 233472 / 2 - 1024 : 232448;
   static constexpr int kRingMax = (kBudget - kFixed) / kBox8;
   static constexpr int kRing = kRingMax > 16 ? 16 : kRingMax;
   static constexpr int kSmem = kRing * kBox8 + kFixed;
   static constexpr int kTmemCols = 6 * kN2 <= 256 ? 256 : 512;   // 2 S^T buffers + 4 O^T chunks
-  static_assert(kRing >= 2 * kNB8, "the ring holds two tiles");
+  // the next tile's boxes are probed by the parity of their full barrier, which
+  // is unambiguous while box c - kRing has been waited for: true up to c =
+  // (first box of this tile) + 2 kNB8 - 1 when kRing >= kNB8
+  static_assert(kRing >= kNB8 + 1, "the ring holds more than one tile");
+  static_assert(kCtasPerSm * kTmemCols <= 512, "tensor memory of the CTAs sharing an SM");
 };
 
 template <int HG>
-__global__ void __launch_bounds__(64 + 128 * (HG >= 32 ? 2 : 1), 1)
+__global__ void __launch_bounds__(64 + 128 * (HG >= 32 ? 2 : 1), (HG == 16 ? 2 : 1))
     decode_attn_fp8_kernel(const __grid_constant__ DecodeArgs a) {
   using C = Dec8Cfg<HG>;
   constexpr int NR = C::kRing, N2 = C::kN2;
@@ -399,7 +426,7 @@ __global__ void __launch_bounds__(64 + 128 * (HG >= 32 ? 2 : 1), 1)
           float x[16];
           load16(c, x);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) need |= x[j] > m[c + j] + 8.f;
+          for (int j = 0; j < 16; ++j) need |= x[j] > m[c + j] + kRaise8;
         }
         const int par = ntile & 1;
         const int vslot = static_cast<int>(ntile % 3u);
@@ -455,7 +482,7 @@ __global__ void __launch_bounds__(64 + 128 * (HG >= 32 ? 2 : 1), 1)
             }
           }
         }
-        // P' = 256 exp2(s - m) as a hi + lo e4m3 pair, this thread's token column
+        // P' = kPScale exp2(s - m) as a hi + lo e4m3 pair, this thread's token column
         // of P [2 HG heads x 128 tokens] (K-major, 128-byte swizzle)
 #pragma unroll
         for (int c = 0; c < HT; c += 16) {

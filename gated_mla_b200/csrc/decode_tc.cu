@@ -869,7 +869,8 @@ DecodeLayout decode_layout(int B, int H, int eff_heads, int d_h, int d_c, int d_
   L.HG = E <= 16 ? 16 : (E % 64 == 0 ? 64 : (E % 32 == 0 ? 32 : 16));
   if (fp8 && L.HG > 32) L.HG = 32;   // hi and lo columns of 64 heads would not fit tensor memory
   L.n_hg = (E + L.HG - 1) / L.HG;
-  L.G = num_sms / L.n_hg;
+  // the FP8 kernel with 16 heads runs two CTAs per SM
+  L.G = ((fp8 && L.HG == 16) ? 2 : 1) * num_sms / L.n_hg;
   if (L.G < 1) L.G = 1;
   L.max_seg = L.G + B + 1;
   const size_t row = static_cast<size_t>(d_c + d_rope);
