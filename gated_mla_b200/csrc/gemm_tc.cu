@@ -536,8 +536,9 @@ SwapPlan gemm_swap_plan(int wtiles, int T, int K, int num_sms) {
   // With a long K (each split keeps >= 16 K blocks at two CTAs per SM), two
   // CTAs per SM keep more weight streams in flight; a short K would only add
   // reduction work.
-  const int slots = tiles <= num_sms ? ((2 * num_sms / tiles) * 16 <= num_kb ? 2 * num_sms : num_sms)
-                                     : 2 * num_sms;
+  const int slots = tiles > num_sms ? 2 * num_sms
+                    : tiles > 0 && (2 * num_sms / tiles) * 16 <= num_kb ? 2 * num_sms
+                                                                        : num_sms;
   int splits = 1;
   if (tiles > 0) splits = tiles <= slots ? slots / tiles : (4 * slots + tiles - 1) / tiles;
   const int max_splits = num_kb / 4 > 1 ? num_kb / 4 : 1;   // keep >= 4 K blocks per split
