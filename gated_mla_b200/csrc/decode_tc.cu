@@ -7,8 +7,8 @@
 //   o^(h)     = W_v^(h) O_lat;   out = sigmoid(g) ⊙ o   (W_v absorbed on the output side)
 //
 // Kernels, in launch order (the W_v product with the gate is a GEMM of gemm_tc.cu):
-//   1. decode_absorb_plan  q_lat = W_k^T q (times scale*log2 e), bf16, with q^R
-//                       appended; its last block splits the cached tokens of all
+//   1. decode_absorb_tc q_lat = W_k^T q (times scale*log2 e) on tcgen05, bf16, with
+//                       q^R appended; its last block splits the cached tokens of all
 //                       sequences into equal per-CTA ranges of 128-token tiles
 //                       (segments).
 //   2. decode_attn      per (CTA range, head group of HG heads): TMA streams the
@@ -140,122 +140,157 @@ __device__ void decode_plan_block(const DecodeArgs& a) {
 
 // ---------------------------------------------------------------------------
 // 2. absorb: qa[b, h, :d_c] = bf16(q_scale * W_k^(h)T q^(h)), qa[b, h, d_c:] = bf16(q_scale * q^R)
-//    One block per (head, 8 sequences, 64 latent columns); the d_h sum is split
-//    over 16 thread groups and reduced in shared memory. The last block of the
-//    grid runs the split plan instead.
+//    On tcgen05, one CTA per (head, 128 latent columns, chunk of up to 128
+//    sequences): q_lat^T = W_k^(h)T q^T with M = 128 latent columns (A = W_k^(h),
+//    MN-major: its rows are d_h, latent columns contiguous), N = sequences (B = q,
+//    K-major), K = d_h, the accumulator in TMEM. W_k is a weight that no kernel
+//    writes, so its boxes are requested before waiting for the queries. The last
+//    CTA of the grid runs the split plan instead.
 // ---------------------------------------------------------------------------
-constexpr int kAbsorbB = 8;
-constexpr int kAbsorbCols = 64;
-constexpr int kAbsorbKG = 16;
+constexpr int kAbsorbM = 128;     // latent columns per CTA
 
-__global__ void __launch_bounds__(256, 4) decode_absorb_plan_kernel(DecodeArgs a) {
+struct AbsorbSmem {
+  uint64_t full, mma_done;
+  uint32_t tmem;
+  int abort;
+  int slot[128];
+  float on[128];
+};
+
+size_t absorb_smem_bytes(int d_h, int bn) {
+  return static_cast<size_t>(2 * d_h * 128 + (d_h / 64) * bn * 128) + 1024 + sizeof(AbsorbSmem);
+}
+
+__global__ void __launch_bounds__(128) decode_absorb_tc_kernel(const __grid_constant__ DecodeArgs a) {
   if (threadIdx.x == 0) griddep_launch_dependents();
-  const int n_cblk = a.d_c / kAbsorbCols;
-  const int n_bblk = (a.B + kAbsorbB - 1) / kAbsorbB;
-  const int blk = blockIdx.x;
-  if (blk == a.H * n_bblk * n_cblk) {
-    griddep_wait();
-    decode_plan_block(a);
+  const int n_ct = a.d_c / kAbsorbM;
+  if (static_cast<int>(blockIdx.x) == a.H * n_ct) {
+    if (blockIdx.y == 0) {
+      griddep_wait();
+      decode_plan_block(a);
+    }
     return;
   }
-  const int h = blk / (n_bblk * n_cblk);
-  const int rem = blk % (n_bblk * n_cblk);
-  const int b0 = (rem / n_cblk) * kAbsorbB;
-  const int cb = rem % n_cblk;
-  const int nb = min(kAbsorbB, a.B - b0);
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int BN = a.absorb_bn;
+  const int nkb = a.d_h / 64;
+  uint8_t* sA = smem;                                  // 2 boxes [d_h rows][64 latent columns]
+  uint8_t* sB = sA + 2 * a.d_h * 128;                  // nkb boxes [BN sequences][64 of d_h]
+  AbsorbSmem* sm = reinterpret_cast<AbsorbSmem*>(sB + nkb * BN * 128);
+  volatile int* abort_flag = &sm->abort;
+  const int h = blockIdx.x / n_ct, ct = blockIdx.x % n_ct;
+  const int b0 = blockIdx.y * BN;
+  const int nb = min(BN, a.B - b0);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t tcols = BN <= 32 ? 32 : (BN <= 64 ? 64 : 128);
+  const uint32_t a_bytes = 2u * a.d_h * 128, b_bytes = static_cast<uint32_t>(nkb * BN * 128);
+
+  if (threadIdx.x == 0) {
+    mbar_init(&sm->full, 1);
+    mbar_init(&sm->mma_done, 1);
+    sm->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&sm->tmem, tcols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm->tmem;
+  bool mma_issued = false;   // thread 0
+  if (threadIdx.x == 0) {
+    tma_prefetch_desc(&a.wk_map);
+    tma_prefetch_desc(&a.q_map);
+    mbar_arrive_expect_tx(&sm->full, a_bytes + b_bytes);
+    for (int j = 0; j < 2; ++j)
+      tma_load_2d(&a.wk_map, &sm->full, sA + j * a.d_h * 128, ct * kAbsorbM + j * 64, h * a.d_h, l2_evict_first());
+  }
+  griddep_wait();   // the queries come from the kernel before this one
   const int dq = a.d_h + a.d_rope;
-  const int row = a.d_c + a.d_rope;
-  __shared__ float sq[kAbsorbB][256];
-  __shared__ float red[kAbsorbKG][kAbsorbB][kAbsorbCols];
-  const int kg = threadIdx.x >> 4;             // 16 groups over d_h
-  const int cl = (threadIdx.x & 15) * 4;       // 4 columns of the block's 64
-  const int c0 = cb * kAbsorbCols + cl;
-  const int kper = (a.d_h + kAbsorbKG - 1) / kAbsorbKG;
-  const __nv_bfloat16* Wk = static_cast<const __nv_bfloat16*>(a.W_k) + static_cast<int64_t>(h) * a.d_h * a.d_c;
-  const int k_lo = kg * kper, k_hi = min(a.d_h, k_lo + kper);
-  // W_k is a weight (no kernel writes it): the first rows of this thread's
-  // slice are in flight before waiting for the kernel that produces the queries
-  constexpr int kChunk = 8;   // rows of W_k held in registers at a time
-  uint2 wv[kChunk];
-  auto load_w = [&](int k0) {
-#pragma unroll
-    for (int i = 0; i < kChunk; ++i)
-      if (k0 + i < k_hi) wv[i] = *reinterpret_cast<const uint2*>(Wk + static_cast<int64_t>(k0 + i) * a.d_c + c0);
-  };
-  load_w(k_lo);
-  griddep_wait();
+  if (threadIdx.x == 0) {
+    for (int kb = 0; kb < nkb; ++kb)
+      tma_load_2d(&a.q_map, &sm->full, sB + kb * BN * 128, h * dq + kb * 64, b0, l2_evict_last());
+  }
   // with hard / quantised gates each sequence stores its heads by slot (heads
   // whose gate is 0 last, their rows zero); otherwise slot = head
-  __shared__ int s_slot[kAbsorbB];
-  __shared__ float s_on[kAbsorbB];
-  if (threadIdx.x < kAbsorbB) {
+  if (threadIdx.x < nb) {
     int slot = h;
     float on = 1.f;
-    const int bi = threadIdx.x;
-    if (a.gate_hard && bi < nb) {
-      const float* z = a.gate_logits + static_cast<int64_t>(b0 + bi) * a.H;
+    const int b = b0 + threadIdx.x;
+    if (a.gate_hard) {
+      const float* z = a.gate_logits + static_cast<int64_t>(b) * a.H;
       int na = 0;
       slot = head_slot(z, a.H, h, a.gate_mode, a.gate_topk, &na);
       const float gv = head_gate(z, a.H, h, a.gate_mode, a.gate_topk);
       on = gv != 0.f ? 1.f : 0.f;
-      if (cb == 0) {
-        a.gvals[static_cast<int64_t>(b0 + bi) * a.H + h] = gv;
-        a.head_of_slot[static_cast<int64_t>(b0 + bi) * a.H + slot] = h;
+      if (ct == 0) {
+        a.gvals[static_cast<int64_t>(b) * a.H + h] = gv;
+        a.head_of_slot[static_cast<int64_t>(b) * a.H + slot] = h;
       }
     }
-    s_slot[bi] = slot;
-    s_on[bi] = on;
+    sm->slot[threadIdx.x] = slot;
+    sm->on[threadIdx.x] = on;
   }
-  const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(a.q);
-  for (int i = threadIdx.x; i < kAbsorbB * a.d_h; i += blockDim.x) {
-    const int bi = i / a.d_h, k = i % a.d_h;
-    sq[bi][k] = bi < nb ? __bfloat162float(q[(static_cast<int64_t>(b0 + bi) * a.H + h) * dq + k]) : 0.f;
+  if (threadIdx.x == 0) {
+    if (mbar_wait(&sm->full, 0, abort_flag, a.status)) {
+      tc_fence_after();
+      // A (MN-major): the two 64-column boxes are d_h * 128 bytes apart; a K step
+      // of 16 rows advances 2 KB. B (K-major): box kb holds d_h columns
+      // [64 kb, 64 kb + 64); a K step of 16 inside a box advances 32 bytes.
+      const uint32_t idesc = idesc_bf16_f32(128, BN, true, false);
+      const uint64_t dA = sdesc_sw128(smem_u32(sA), a.d_h * 128, 1024);
+      const uint64_t dB = sdesc_sw128(smem_u32(sB), 16, 1024);
+      for (int k = 0; k < a.d_h / 16; ++k)
+        umma_bf16(tmem, dA + (k * 2048) / 16, dB + ((k >> 2) * BN * 128 + (k & 3) * 32) / 16, idesc, k != 0);
+      umma_commit(&sm->mma_done);
+      mma_issued = true;
+    } else {
+      mbar_drain(&sm->full, 0);   // copies still in flight land before the block leaves
+    }
   }
   __syncthreads();
-  float acc[kAbsorbB][4];
+  // epilogue: warp w holds latent columns ct*128 + 32 w + lane, one TMEM column per sequence
+  bool ok = !*abort_flag && mbar_wait(&sm->mma_done, 0, abort_flag, a.status);
+  ok = __all_sync(0xffffffffu, ok);
+  if (ok) {
+    tc_fence_after();
+    const int row = a.d_c + a.d_rope;
+    const int c = ct * kAbsorbM + 32 * warp + lane;
+    __nv_bfloat16* qa = static_cast<__nv_bfloat16*>(a.qa);
+    const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * warp) << 16);
+    for (int n0 = 0; n0 < BN; n0 += 16) {
+      uint32_t v[16];
+      tmem_ld16(taddr + n0, v);
+      tmem_ld_wait();
 #pragma unroll
-  for (int bi = 0; bi < kAbsorbB; ++bi)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) acc[bi][j] = 0.f;
-  for (int k0 = k_lo; k0 < k_hi; k0 += kChunk) {
-    if (k0 != k_lo) load_w(k0);
-#pragma unroll
-    for (int i = 0; i < kChunk; ++i) {
-      if (k0 + i >= k_hi) break;
-      const __nv_bfloat162 w01 = *reinterpret_cast<const __nv_bfloat162*>(&wv[i].x);
-      const __nv_bfloat162 w23 = *reinterpret_cast<const __nv_bfloat162*>(&wv[i].y);
-      const float w[4] = {__low2float(w01), __high2float(w01), __low2float(w23), __high2float(w23)};
-#pragma unroll
-      for (int bi = 0; bi < kAbsorbB; ++bi) {
-        const float qk = sq[bi][k0 + i];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[bi][j] = fmaf(qk, w[j], acc[bi][j]);
+      for (int j = 0; j < 16; ++j) {
+        const int n = n0 + j;
+        if (n < nb)
+          qa[(static_cast<int64_t>(b0 + n) * a.H + sm->slot[n]) * row + c] =
+              __float2bfloat16_rn(__uint_as_float(v[j]) * a.q_scale * sm->on[n]);
       }
     }
-  }
-#pragma unroll
-  for (int bi = 0; bi < kAbsorbB; ++bi)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) red[kg][bi][cl + j] = acc[bi][j];
-  __syncthreads();
-  __nv_bfloat16* qa = static_cast<__nv_bfloat16*>(a.qa);
-  for (int o = threadIdx.x; o < kAbsorbB * kAbsorbCols; o += blockDim.x) {
-    const int bi = o / kAbsorbCols, c = o % kAbsorbCols;
-    if (bi >= nb) continue;
-    float v = 0.f;
-#pragma unroll
-    for (int g = 0; g < kAbsorbKG; ++g) v += red[g][bi][c];
-    qa[(static_cast<int64_t>(b0 + bi) * a.H + s_slot[bi]) * row + cb * kAbsorbCols + c] =
-        __float2bfloat16_rn(v * a.q_scale * s_on[bi]);
-  }
-  // decoupled RoPE query dims: copied (already rotated), scaled
-  if (cb == 0) {
-    for (int i = threadIdx.x; i < nb * a.d_rope; i += blockDim.x) {
-      const int bi = i / a.d_rope, r = i % a.d_rope;
-      const int64_t src = (static_cast<int64_t>(b0 + bi) * a.H + h) * dq + a.d_h + r;
-      qa[(static_cast<int64_t>(b0 + bi) * a.H + s_slot[bi]) * row + a.d_c + r] =
-          __float2bfloat16_rn(__bfloat162float(q[src]) * a.q_scale * s_on[bi]);
+    // decoupled RoPE query dims: copied (already rotated), scaled
+    if (ct == 0) {
+      const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(a.q);
+      for (int i = threadIdx.x; i < nb * a.d_rope; i += blockDim.x) {
+        const int n = i / a.d_rope, r = i % a.d_rope;
+        const int64_t src = (static_cast<int64_t>(b0 + n) * a.H + h) * dq + a.d_h + r;
+        qa[(static_cast<int64_t>(b0 + n) * a.H + sm->slot[n]) * row + a.d_c + r] =
+            __float2bfloat16_rn(__bfloat162float(q[src]) * a.q_scale * sm->on[n]);
+      }
     }
+  } else if (mma_issued) {
+    mbar_drain(&sm->mma_done, 0);   // an issued product completes before TMEM is freed
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, tcols);
   }
 }
 
@@ -938,11 +973,17 @@ static cudaError_t launch_decode_fp8(DecodeArgs& a, cudaStream_t st) {
   return e;
 }
 
+int absorb_tile_n(int B) { return B >= 128 ? 128 : ((B + 15) / 16) * 16; }
+
 cudaError_t launch_decode_bf16(DecodeArgs& a, cudaStream_t st) {
   if (a.fp8) return launch_decode_fp8(a, st);
-  const int n_absorb = a.H * ((a.B + kAbsorbB - 1) / kAbsorbB) * (a.d_c / kAbsorbCols);
+  const size_t smem = absorb_smem_bytes(a.d_h, a.absorb_bn);
+  cudaError_t e = cudaFuncSetAttribute(decode_absorb_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
   prof_begin(st, "decode_absorb_plan");
-  cudaError_t e = launch_pdl(decode_absorb_plan_kernel, dim3(n_absorb + 1), dim3(256), 0, st, 1, a);
+  e = launch_pdl(decode_absorb_tc_kernel, dim3(a.H * (a.d_c / kAbsorbM) + 1, (a.B + a.absorb_bn - 1) / a.absorb_bn),
+                 dim3(128), smem, st, 1, a);
   prof_end(st);
   if (e != cudaSuccess) return e;
   const int nbox = (a.d_c + a.d_rope) / 64;

@@ -633,6 +633,17 @@ static gmla_status decode_impl(const gmla_config* cfg, const gmla_weights* w, co
           : !make_tmap_2d(&a.qa_map, ws + L.off_qa, row, static_cast<uint64_t>(B) * cfg->n_heads,
                           static_cast<uint64_t>(row) * 2, 64, L.HG, true))
     return fail(GMLA_ERR_CUDA, "tensor map for the absorbed queries failed");
+  if (!fp8) {
+    // the tensor-core absorb: W_k as [H*d_h, d_c] in boxes of [d_h x 64], the
+    // queries as [B, H*(d_h + d_R)] in boxes of [absorb_bn x 64]
+    const int dq = cfg->d_h + cfg->d_rope;
+    a.absorb_bn = absorb_tile_n(B);
+    if (!make_tmap_2d(&a.wk_map, w->W_k, cfg->d_c, static_cast<uint64_t>(cfg->n_heads) * cfg->d_h,
+                      static_cast<uint64_t>(cfg->d_c) * 2, 64, cfg->d_h, true) ||
+        !make_tmap_2d(&a.q_map, q, static_cast<uint64_t>(cfg->n_heads) * dq, B,
+                      static_cast<uint64_t>(cfg->n_heads) * dq * 2, 64, a.absorb_bn, true))
+      return fail(GMLA_ERR_CUDA, "tensor maps for the query absorption failed");
+  }
   a.cache = cv;
   a.seq_lens = seq_lens;
   a.q = q;

@@ -61,6 +61,9 @@ SwapPlan gemm_swap_plan(int wtiles, int T, int K, int num_sms);
 struct DecodeArgs {
   CUtensorMap cache_map;     // contiguous: 2D [B*cap, row]; paged: 3D [pages, page_size, row]
   CUtensorMap qa_map;        // 2D [B*H, row] bf16 absorbed queries
+  CUtensorMap wk_map;        // 2D [H*d_h, d_c] bf16 W_k, boxes of [d_h rows x 64 columns] (bf16 cache)
+  CUtensorMap q_map;         // 2D [B, H*(d_h + d_R)] bf16 queries, boxes of [absorb_bn rows x 64] (bf16 cache)
+  int32_t absorb_bn;         // sequences per absorb CTA (multiple of 16, <= 128)
   CacheView cache;
   const int32_t* seq_lens;   // [B]
   const void* q;             // [B, H, d_h + d_R]
@@ -123,6 +126,8 @@ struct DecodeLayout {
 // eff_heads: the most heads a sequence attends with (H, or k with top-k gates),
 // which sets the head groups of the attention kernel.
 DecodeLayout decode_layout(int B, int H, int eff_heads, int d_h, int d_c, int d_rope, int num_sms, bool fp8 = false);
+// sequences per CTA of the tensor-core absorb (N of its MMA)
+int absorb_tile_n(int B);
 cudaError_t launch_decode_bf16(DecodeArgs& a, cudaStream_t st);
 
 // ----- fp32 CUDA-core path (simt_f32.cu) -----
