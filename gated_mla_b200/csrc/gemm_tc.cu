@@ -533,14 +533,16 @@ SwapPlan gemm_swap_plan(int wtiles, int T, int K, int num_sms) {
   // Few tiles: split K (one cluster of splits per tile) until the tiles fill one
   // CTA per SM. Many tiles: split so there are at least four waves of two CTAs
   // per SM (tail imbalance < 25%).
-  // With a long K (each split keeps >= 16 K blocks at two CTAs per SM), two
-  // CTAs per SM keep more weight streams in flight; a short K would only add
-  // reduction work.
-  const int slots = tiles > num_sms ? 2 * num_sms
-                    : tiles > 0 && (2 * num_sms / tiles) * 16 <= num_kb ? 2 * num_sms
-                                                                        : num_sms;
+  // With a long K (each split would keep >= 16 K blocks at two CTAs per SM), about
+  // 1.5 CTAs per SM: more weight streams in flight than one per SM, while every
+  // CTA still finds a slot as the kernel before it drains, so all of them request
+  // their weight tiles early (measured faster than two per SM on a 56-tile,
+  // K = 16384 output projection); a short K would only add reduction work.
   int splits = 1;
-  if (tiles > 0) splits = tiles <= slots ? slots / tiles : (4 * slots + tiles - 1) / tiles;
+  if (tiles > num_sms)
+    splits = (8 * num_sms + tiles - 1) / tiles;
+  else if (tiles > 0)
+    splits = (2 * num_sms / tiles) * 16 <= num_kb ? (3 * num_sms / 2 + tiles - 1) / tiles : num_sms / tiles;
   const int max_splits = num_kb / 4 > 1 ? num_kb / 4 : 1;   // keep >= 4 K blocks per split
   splits = splits < 1 ? 1 : (splits > max_splits ? max_splits : splits);
   if (splits > 8) splits = 8;   // the splits of a tile form one (portable-size) cluster

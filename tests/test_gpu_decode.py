@@ -79,6 +79,14 @@ def test_decode_heads_not_multiple_of_16():
     _check(inp, run_decode(inp))
 
 
+def test_decode_more_than_128_sequences():
+    """136 sequences: the query absorption takes its sequences in chunks of 128
+    (the second chunk ragged), each chunk one column block of its MMA."""
+    lens = [1 + (37 * b) % 300 for b in range(136)]
+    inp = small_decode("decode_b32", 136, lens, n_heads=4, d_model=256)
+    _check(inp, run_decode(inp), check_cache=False)
+
+
 def test_decode_many_segments_per_sequence():
     """One long sequence spread over every CTA (split-K merge across ~148 partials)."""
     inp = small_decode("decode_b32", 2, [40000, 3])
