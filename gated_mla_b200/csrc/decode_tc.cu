@@ -428,6 +428,20 @@ __global__ void __launch_bounds__(64 + 128 * (HG >= 32 ? 2 : 1), 1) decode_attn_
       for (int t = sg.y; t < sg.z && ok; ++t) {
         const int tok0 = t * kTileTok;
         const int valid = min(kTileTok, L - tok0);
+        if (C::kRing == kNcBox && !paged && t + 1 < sg.z) {
+          // A ring of one tile: each tile's boxes are requested only as the previous
+          // weighted sum frees their slots, so the next tile's rows (contiguous in
+          // the cache) are brought into L2 now, in NBOX pieces, one per lane.
+          const int rows_next = min(kTileTok, L - tok0 - kTileTok);
+          const uint32_t row_bytes = static_cast<uint32_t>(a.cache.row) * 2;
+          const uint32_t total = static_cast<uint32_t>(rows_next) * row_bytes;   // a multiple of 16
+          const uint32_t piece = ((total + NBOX - 1) / NBOX + 15) & ~15u;
+          const uint32_t off = static_cast<uint32_t>(lane) * piece;
+          if (lane < NBOX && off < total)
+            bulk_prefetch_l2(static_cast<const uint8_t*>(a.cache.data) +
+                                 (static_cast<int64_t>(b) * a.cache.capacity + tok0 + kTileTok) * row_bytes + off,
+                             min(piece, total - off));
+        }
         const int nchunk = ps >= kTileTok ? 1 : (valid + ps - 1) / ps;   // <= 16 (page size >= 8)
         int page = 0;
         if (paged && lane < nchunk)

@@ -163,6 +163,12 @@ __device__ __forceinline__ float sigmoid_tanh(float x) {
   return fmaf(0.5f, t, 0.5f);
 }
 // Bring the line holding `p` into L2 (no result, no fault on any address).
+// Asynchronous prefetch of `bytes` bytes (a multiple of 16, from a 16-byte
+// aligned address) of global memory into L2; no shared memory is written.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(bytes)
+               : "memory");
+}
 __device__ __forceinline__ void prefetch_l2(const void* p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
