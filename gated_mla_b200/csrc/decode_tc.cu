@@ -76,13 +76,19 @@ __device__ __forceinline__ int seq_tiles(int L, int start) {
 // Tiles of 128 tokens of all sequences, concatenated, are cut into G equal
 // ranges (one per CTA of a head group). A segment is the part of one sequence
 // inside one range; seg_info = {sequence, first tile, end tile, CTA}.
+// A CTA pays about one tile's time for each segment it starts (the partial of
+// the previous one written, the next absorbed queries loaded). So when the CTAs
+// average at least 4 tiles, each sequence's range is preceded by one virtual
+// tile: a range that crosses a sequence start holds one real tile fewer. (With
+// ranges of >= 2 units and no two virtual units adjacent, every range still
+// holds a real tile.)
 __device__ void decode_plan_block(const DecodeArgs& a) {
   __shared__ int s_warp[32];
   __shared__ int s_total;
-  __shared__ int s_sum;
+  __shared__ int s_sum, s_nz;
   const int tid = threadIdx.x;
   const int limit = a.cache.paged ? a.cache.max_pages_per_seq * a.cache.page_size : a.cache.capacity;
-  if (tid == 0) s_sum = 0;
+  if (tid == 0) s_sum = s_nz = 0;
   __syncthreads();
   for (int b = tid; b < a.B; b += blockDim.x) {
     int L = a.seq_lens[b];
@@ -91,12 +97,16 @@ __device__ void decode_plan_block(const DecodeArgs& a) {
       report_status(a.status, kStatusRange);
       L = 0;
     }
-    atomicAdd(&s_sum, seq_tiles(L, s0));
+    const int t = seq_tiles(L, s0);
+    atomicAdd(&s_sum, t);
+    if (t > 0) atomicAdd(&s_nz, 1);
   }
   __syncthreads();
   const int total = s_sum;
-  const int tpc = total > 0 ? (total + a.G - 1) / a.G : 1;
-  int tile_carry = 0, seg_carry = 0;
+  const int vu = total >= 4 * a.G ? 1 : 0;        // virtual units before each sequence with tiles
+  const int total_u = total + vu * s_nz;
+  const int tpc = total_u > 0 ? (total_u + a.G - 1) / a.G : 1;
+  int unit_carry = 0, seg_carry = 0;
   for (int base = 0; base < a.B; base += blockDim.x) {
     const int b = base + tid;
     int L = b < a.B ? a.seq_lens[b] : 0;
@@ -104,13 +114,14 @@ __device__ void decode_plan_block(const DecodeArgs& a) {
     if (L < 0 || L > limit || b >= a.cache.batch || s0 < 0) L = 0;
     const int t = seq_tiles(L, s0);
     const int ts = s0 / kTileTok;   // first tile of the sequence's range
-    int tsum, ssum;
-    const int P = tile_carry + block_excl_scan(t, s_warp, &s_total);
-    tsum = s_total;
+    int usum, ssum;
+    const int P = unit_carry + block_excl_scan(t > 0 ? t + vu : 0, s_warp, &s_total);   // first unit
+    usum = s_total;
+    const int Q = P + vu;           // unit of the sequence's first tile
     int nseg = 0, g_first = 0;
     if (t > 0) {
-      g_first = P / tpc;
-      nseg = (P + t - 1) / tpc - g_first + 1;
+      g_first = Q / tpc;
+      nseg = (Q + t - 1) / tpc - g_first + 1;
     }
     const int S = seg_carry + block_excl_scan(nseg, s_warp, &s_total);
     ssum = s_total;
@@ -118,16 +129,16 @@ __device__ void decode_plan_block(const DecodeArgs& a) {
       a.seq_first_seg[b] = S;
       for (int k = 0; k < nseg; ++k) {
         const int g = g_first + k;
-        const int lo = max(P, g * tpc), hi = min(P + t, (g + 1) * tpc);
-        a.seg_info[S + k] = make_int4(b, ts + lo - P, ts + hi - P, g);
-        if (g * tpc >= P) a.cta_first_seg[g] = S + k;   // range g starts inside sequence b
+        const int lo = max(Q, g * tpc), hi = min(Q + t, (g + 1) * tpc);
+        a.seg_info[S + k] = make_int4(b, ts + lo - Q, ts + hi - Q, g);
+        if (g * tpc >= P) a.cta_first_seg[g] = S + k;   // range g starts inside sequence b's units
       }
     }
-    tile_carry += tsum;
+    unit_carry += usum;
     seg_carry += ssum;
   }
   if (tid == 0) a.seq_first_seg[a.B] = seg_carry;
-  const int g_used = total > 0 ? (total - 1) / tpc + 1 : 0;
+  const int g_used = total_u > 0 ? (total_u - 1) / tpc + 1 : 0;
   for (int g = g_used + tid; g <= a.G; g += blockDim.x) a.cta_first_seg[g] = seg_carry;
   if (a.gate_hard) {   // heads of each sequence whose gate is not 0
     for (int b = tid; b < a.B; b += blockDim.x) {
