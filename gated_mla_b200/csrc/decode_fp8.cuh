@@ -261,7 +261,7 @@ __global__ void __launch_bounds__(64 + 128 * (HG >= 32 ? 2 : 1), (HG == 16 ? 2 :
     for (int si = seg_lo; si < seg_hi && ok; ++si) {
       const int4 sg = a.seg_info[si];
       const int b = sg.x;
-      const int L = a.seq_lens[b];
+      const int L = sg.w;
       if (seg_heads(a, b, hg, heads_valid) == 0) continue;
       if (lane == 0) {
         if (nq > 0 && !mbar_wait(&sm->q_empty, (nq - 1) & 1, abort_flag, a.status)) ok = false;
@@ -392,7 +392,7 @@ __global__ void __launch_bounds__(64 + 128 * (HG >= 32 ? 2 : 1), (HG == 16 ? 2 :
     for (int si = seg_lo; si < seg_hi; ++si) {
       const int4 sg = a.seg_info[si];
       const int b = sg.x;
-      const int L = a.seq_lens[b];
+      const int L = sg.w;
       const int S0 = a.seq_starts ? a.seq_starts[b] : 0;
       const int hv = seg_heads(a, b, hg, heads_valid);
       if (hv == 0) continue;

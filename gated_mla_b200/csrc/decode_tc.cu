@@ -75,13 +75,15 @@ __device__ __forceinline__ int seq_tiles(int L, int start) {
 
 // Tiles of 128 tokens of all sequences, concatenated, are cut into G equal
 // ranges (one per CTA of a head group). A segment is the part of one sequence
-// inside one range; seg_info = {sequence, first tile, end tile, CTA}.
-// A CTA pays about one tile's time for each segment it starts (the partial of
-// the previous one written, the next absorbed queries loaded). So when the CTAs
-// average at least 4 tiles, each sequence's range is preceded by one virtual
-// tile: a range that crosses a sequence start holds one real tile fewer. (With
-// ranges of >= 2 units and no two virtual units adjacent, every range still
-// holds a real tile.)
+// inside one range; seg_info = {sequence, first tile, end tile, sequence length}
+// (the length carried along saves the attention kernel a dependent load).
+// A CTA pays about one to two tiles' time for each segment it starts (the
+// partial of the previous one written, the next absorbed queries loaded; more
+// tiles' worth where tiles are cheap, as with the FP8 cache). So when the CTAs
+// average at least 4 tiles, each sequence's range is preceded by two virtual
+// tiles: a range that crosses a sequence start holds two real tiles fewer.
+// (Ranges then span >= 4 units and the virtual runs 2, each followed by a real
+// tile, so every range still holds a real tile.)
 __device__ void decode_plan_block(const DecodeArgs& a) {
   __shared__ int s_warp[32];
   __shared__ int s_total;
@@ -103,7 +105,7 @@ __device__ void decode_plan_block(const DecodeArgs& a) {
   }
   __syncthreads();
   const int total = s_sum;
-  const int vu = total >= 4 * a.G ? 1 : 0;        // virtual units before each sequence with tiles
+  const int vu = total >= 4 * a.G ? 2 : 0;        // virtual units before each sequence with tiles
   const int total_u = total + vu * s_nz;
   const int tpc = total_u > 0 ? (total_u + a.G - 1) / a.G : 1;
   int unit_carry = 0, seg_carry = 0;
@@ -130,7 +132,7 @@ __device__ void decode_plan_block(const DecodeArgs& a) {
       for (int k = 0; k < nseg; ++k) {
         const int g = g_first + k;
         const int lo = max(Q, g * tpc), hi = min(Q + t, (g + 1) * tpc);
-        a.seg_info[S + k] = make_int4(b, ts + lo - Q, ts + hi - Q, g);
+        a.seg_info[S + k] = make_int4(b, ts + lo - Q, ts + hi - Q, L);
         if (g * tpc >= P) a.cta_first_seg[g] = S + k;   // range g starts inside sequence b's units
       }
     }
@@ -423,7 +425,7 @@ __global__ void __launch_bounds__(64 + 128 * (HG >= 32 ? 2 : 1), 1) decode_attn_
     for (int si = seg_lo; si < seg_hi && ok; ++si) {
       const int4 sg = a.seg_info[si];
       const int b = sg.x;
-      const int L = a.seq_lens[b];
+      const int L = sg.w;
       if (seg_heads(a, b, hg, heads_valid) == 0) continue;
       if (lane == 0) {
         if (nq > 0 && !mbar_wait(&sm->q_empty, (nq - 1) & 1, abort_flag, a.status)) ok = false;
@@ -610,7 +612,7 @@ __global__ void __launch_bounds__(64 + 128 * (HG >= 32 ? 2 : 1), 1) decode_attn_
     bool ok = true;
     for (int si = seg_lo; si < seg_hi; ++si) {
       const int4 sg = a.seg_info[si];
-      const int L = a.seq_lens[sg.x];
+      const int L = sg.w;
       const int S0 = a.seq_starts ? a.seq_starts[sg.x] : 0;
       const int hv = seg_heads(a, sg.x, hg, heads_valid);
       if (hv == 0) continue;

@@ -74,7 +74,7 @@ struct DecodeArgs {
   void* qa;                  // workspace: [B*H, row] bf16
   float* o_part;             // workspace: [n_hg, max_seg, HG, d_c]
   float* ml_part;            // workspace: [n_hg, max_seg, HG, 2]
-  int4* seg_info;            // workspace: [max_seg]
+  int4* seg_info;            // workspace: [max_seg] {sequence, first tile, end tile, length}
   int32_t* seq_first_seg;    // workspace: [B + 1]
   int32_t* cta_first_seg;    // workspace: [G + 1]
   void* olat;                // workspace: [H, B, d_c] bf16 merged latent outputs
