@@ -63,3 +63,18 @@ def test_context_parallel_with_hard_top_k_gates():
     o, gpu = _emulate(inp, 2)
     ref = oracle.decode(oracle.params(inp), inp["x"], inp["past"])
     assert_close(o, ref["gated"], BF16_TOL, "gated o")
+
+
+def test_context_parallel_long_shares():
+    """Two sequences of 76,800 rows: the whole cache and each rank's share hold
+    enough 128-token tiles (600 per share) that the split plan charges each
+    sequence start its virtual tiles, in the partial decode as in the whole one.
+    The oracle checks sequence 0 in the absorbed form (pinned equal to the
+    explicit form by the oracle's tests)."""
+    inp = small_decode("decode_b32", 2, [76800, 76800])
+    o, gpu = _emulate(inp, 2)
+    assert np.all(np.isfinite(o))
+    m = metrics(o, gpu["o"])
+    assert m["rel_l2"] < 3e-3, m
+    ref = oracle.decode(oracle.params(inp), inp["x"], inp["past"], seqs=[0], absorbed=True)
+    assert_close(o[[0]], ref["gated"], BF16_TOL, "gated o, sequence 0")
