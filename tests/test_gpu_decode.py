@@ -79,6 +79,13 @@ def test_decode_heads_not_multiple_of_16():
     _check(inp, run_decode(inp))
 
 
+def test_decode_head_dim_256():
+    """d_h = 256: the query absorption takes W_k^(h) in boxes of 256 rows and K = 256
+    (16 MMAs), and the W_v product spans two 128-row tiles per head."""
+    inp = small_decode("decode_b32", 3, [5, 130, 700], n_heads=4, d_h=256, d_model=512)
+    _check(inp, run_decode(inp))
+
+
 def test_decode_more_than_128_sequences():
     """136 sequences: the query absorption takes its sequences in chunks of 128
     (the second chunk ragged), each chunk one column block of its MMA."""
