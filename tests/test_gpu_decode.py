@@ -58,10 +58,13 @@ def test_decode_paged_per_head_gate():
     _check(inp, run_decode(inp))
 
 
-def test_decode_paged_equals_contiguous():
+@pytest.mark.parametrize("page_size", [16, 64, 128, 256])
+def test_decode_paged_equals_contiguous(page_size):
+    """Pages smaller than a 128-token tile are copied one per lane; pages of 128 or
+    more hold whole tiles, copied as one box at the tile's offset in the page."""
     inp = small_decode("decode_b32", 4, [65, 300, 1, 1000])
     a = run_decode(inp, paged=False)
-    w = inp["workload"].replace(paged=True, page_size=64)
+    w = inp["workload"].replace(paged=True, page_size=page_size)
     inp2 = dict(inp, workload=w)
     b = run_decode(inp2, paged=True)
     m = metrics(b["o"], a["o"])
